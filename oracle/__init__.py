@@ -1,0 +1,44 @@
+"""CPU oracle for block-sparse video attention -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow, fp64 NumPy restatement of what the block-sparse attention path
+computes, written from the pages' prose:
+
+  * LoSA (abstract, scholarbro.com author page of C. Sun): exact block
+    attention mass measured at one dense step; per head and query block the
+    smallest key/value block set whose retained mass meets a 99% threshold;
+    the frozen block indices reused at later steps.
+  * VMoBA (pith.science review of arXiv 2506.23858, "What carries the
+    argument", referee report major comment 1, circularity check, free
+    parameters): key blocks represented by their mean; global selection over
+    all query-key block pairs of a head; threshold selection keeping the
+    smallest number of pairs whose cumulative normalized similarity reaches
+    tau; the layer-wise 1D-2D-3D block partition; empty query rows.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  It imports nothing from the CUDA library or its
+Python binding and shares no helper with them.
+
+Modules
+  attention   dense_attention, sparse_attention        (pinned)
+  scores      block_mass, meanpool_scores              (pinned)
+  select      select_contract, select_fp64, csr tools  (pinned)
+  partition   raster / 1D / 2D / 3D token orders       (pinned)
+
+Every function is pinned by a ``-m "not gpu"`` test against something other
+than itself (library routines, closed forms, brute force, hand-worked
+examples under ``tests/golden/``); none is "parity unpinned".
+"""
+from .attention import dense_attention, sparse_attention
+from .scores import block_mass, meanpool_scores
+from .select import (select_contract, select_fp64, InvalidScores, threshold_fixed_point,
+                     csr_rows, csr_from_rows)
+from .partition import (perm_raster, perm_1d_temporal, perm_2d_frame_tiles, perm_3d_tiles,
+                        perm_for_call, PARTITION_CYCLE)
+
+__all__ = [
+    "dense_attention", "sparse_attention", "block_mass", "meanpool_scores",
+    "select_contract", "select_fp64", "InvalidScores", "threshold_fixed_point",
+    "csr_rows", "csr_from_rows",
+    "perm_raster", "perm_1d_temporal", "perm_2d_frame_tiles", "perm_3d_tiles",
+    "perm_for_call", "PARTITION_CYCLE",
+]
