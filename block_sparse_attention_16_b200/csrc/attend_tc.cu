@@ -1,0 +1,424 @@
+// Block-sparse flash attention on sm_100a tensor cores (bf16 in, fp32 accumulate).
+//
+// What it computes (VMoBA review on pith.science, "What carries the argument":
+// only the selected key blocks contribute their actual key-value pairs; LoSA
+// abstract: the frozen block indices are reused at every later step):
+//   out_r = sum_{c in K_i} softmax_{c in K_i}(q_r . k_c / sqrt(d)) v_c
+// where K_i is the set of valid keys of the blocks kept for query block i.
+// An empty list gives out_r = 0 and lse_r = -inf.
+//
+// Tiling.  A CTA owns a 128-row query tile (one 128-token block, or two
+// 64-token blocks that share the tile).  It walks the ascending union of the
+// tile's kept key blocks in 64-key steps; a row whose own block did not keep
+// the current key block gives it zero probability.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread t owns tile row t = TMEM lane t.  Reads S from
+//              TMEM, keeps the running max / sum, writes P (bf16) into a
+//              128-byte-swizzled shared-memory tile, rescales O in TMEM when
+//              the running max grows by more than 2^8, and writes the output.
+//   warp 4     TMA producer: Q once, then K and V 64-key tiles through a
+//              3-stage ring.
+//   warp 5     UMMA issuer: S = Q K^T (M=128, N=64, K=d) into one of two TMEM
+//              S buffers, then O += P V (M=128, N=d, K=64) into TMEM.
+// TMEM columns: [0,64) S0, [64,128) S1, [128,128+d) O.
+#include "lbsa_device.cuh"
+
+namespace lbsa {
+namespace {
+
+constexpr int BM = 128;           // query rows per tile
+constexpr int BK = 64;            // keys per step
+constexpr int NS = 3;             // K/V ring depth
+constexpr int kThreads = 192;
+constexpr int kMaxBlocks = 4096;  // nB bound (bitmap size)
+constexpr int kMaxWords = kMaxBlocks / 32;
+constexpr uint32_t kTmemCols = 256;
+
+template <int D>
+struct Layout {
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BK * D * 2;
+  static constexpr int P_BYTES = BM * BK * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int NBAR = 1 + 4 * NS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort, n_entries, pad
+  static constexpr int OFF_BITMAP = OFF_MISC + 16;
+  static constexpr int OFF_SCHED = OFF_BITMAP + 2 * kMaxWords * 4;
+  static size_t bytes(int nB) { return OFF_SCHED + static_cast<size_t>(nB) * 4 + 1024; }
+};
+
+struct Bars {
+  uint64_t* q_full;
+  uint64_t* k_full;
+  uint64_t* k_empty;
+  uint64_t* v_full;
+  uint64_t* v_empty;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_done;
+  uint64_t* drain;
+};
+
+__device__ __forceinline__ Bars make_bars(uint8_t* base) {
+  uint64_t* b = reinterpret_cast<uint64_t*>(base);
+  Bars r;
+  r.q_full = b;
+  r.k_full = b + 1;
+  r.k_empty = b + 1 + NS;
+  r.v_full = b + 1 + 2 * NS;
+  r.v_empty = b + 1 + 3 * NS;
+  r.s_full = b + 1 + 4 * NS;
+  r.p_full = r.s_full + 2;
+  r.o_done = r.p_full + 2;
+  r.drain = r.o_done + 2;
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v, const AttendArgs args, float scale_log2) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int tile = blockIdx.x;
+  const int h = blockIdx.y;
+  const int bb = blockIdx.z;
+  const int nB = args.nB;
+  const int blk = args.block;               // 64 or 128
+  const int spb = blk / BK;                 // steps per kept key block
+
+  Bars bars = make_bars(smem + L::OFF_BAR);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  uint32_t* bm0 = reinterpret_cast<uint32_t*>(smem + L::OFF_BITMAP);
+  uint32_t* bm1 = bm0 + kMaxWords;
+  uint32_t* sched = reinterpret_cast<uint32_t*>(smem + L::OFF_SCHED);
+  const int nwords = (nB + 31) >> 5;
+  // a CTA of this launch already gave up on a wait: skip the work, the call has failed
+  if (*reinterpret_cast<volatile int32_t*>(args.status) == LBSA_ERR_TIMEOUT) return;
+
+  // ---- set-up: barriers, TMEM, schedule (union of the tile's block lists)
+  if (tid == 0) {
+    mbar_init(bars.q_full, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(bars.k_full + i, 1);
+      mbar_init(bars.k_empty + i, 1);
+      mbar_init(bars.v_full + i, 1);
+      mbar_init(bars.v_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars.s_full + i, 1);
+      mbar_init(bars.p_full + i, 128);
+      mbar_init(bars.o_done + i, 1);
+    }
+    mbar_init(bars.drain, 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(misc, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = tid; i < 2 * kMaxWords; i += kThreads) bm0[i] = 0;
+  __syncthreads();
+
+  const int qb0 = (blk == 64) ? 2 * tile : tile;
+  const int qb1 = (blk == 64 && 2 * tile + 1 < nB) ? 2 * tile + 1 : -1;
+  {
+    const long long row0 = (static_cast<long long>(bb) * args.H + h) * nB + qb0;
+    const int c0 = args.counts[row0];
+    const int32_t* l0 = args.cols + row0 * nB;
+    for (int i = tid; i < c0; i += kThreads) {
+      const int c = l0[i];
+      if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
+      else atomicOr(&bm0[c >> 5], 1u << (c & 31));
+    }
+    if (qb1 >= 0) {
+      const long long row1 = row0 + 1;
+      const int c1 = args.counts[row1];
+      const int32_t* l1 = args.cols + row1 * nB;
+      for (int i = tid; i < c1; i += kThreads) {
+        const int c = l1[i];
+        if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
+        else atomicOr(&bm1[c >> 5], 1u << (c & 31));
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // each lane owns a contiguous run of bitmap words; exclusive scan of popcounts
+    const int per = (nwords + 31) / 32;
+    const int w0 = lane * per;
+    int cnt = 0;
+    for (int w = w0; w < w0 + per && w < nwords; ++w) cnt += __popc(bm0[w] | bm1[w]);
+    int incl = cnt;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = incl - cnt;
+    for (int w = w0; w < w0 + per && w < nwords; ++w) {
+      const uint32_t a = bm0[w], b = bm1[w];
+      uint32_t u = a | b;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1;
+        uint32_t mask = (blk == 64) ? (((a >> bit) & 1u) | (((b >> bit) & 1u) << 1)) : 3u;
+        sched[pos++] = static_cast<uint32_t>(w * 32 + bit) | (mask << 30);
+      }
+    }
+    if (lane == 31) misc[2] = static_cast<uint32_t>(incl);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = misc[0];
+  const int n_steps = static_cast<int>(misc[2]) * spb;
+  const long long wl = args.wait_limit;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+      uint8_t* sQ = smem + L::OFF_Q;
+      if (n_steps > 0) {
+        mbar_arrive_expect_tx(bars.q_full, L::Q_BYTES);
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, bars.q_full, c * 64, tile * BM, h, bb);
+      }
+      int issued = 0;
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % NS;
+        const uint32_t ph = (s / NS) & 1;
+        const uint32_t e = sched[s / spb];
+        const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
+        if (s >= NS && !mbar_wait(bars.k_empty + st, ph ^ 1, wl, args.status, abort_flag)) break;
+        uint8_t* sK = smem + L::OFF_K + st * L::KV_BYTES;
+        mbar_arrive_expect_tx(bars.k_full + st, L::KV_BYTES);
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, bars.k_full + st, c * 64, key0, h, bb);
+        if (s >= NS && !mbar_wait(bars.v_empty + st, ph ^ 1, wl, args.status, abort_flag)) { issued = s + 1; break; }
+        uint8_t* sV = smem + L::OFF_V + st * L::KV_BYTES;
+        mbar_arrive_expect_tx(bars.v_full + st, L::KV_BYTES);
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(sV + c * BK * 128, &tmap_v, bars.v_full + st, c * 64, key0, h, bb);
+        issued = s + 1;
+      }
+      if (*abort_flag) {
+        // let copies still in flight land before the CTA can exit
+        for (int s = (issued > NS ? issued - NS : 0); s < issued; ++s) {
+          mbar_wait(bars.k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
+          mbar_wait(bars.v_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(BM, BK, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(BM, D, 1);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+      const uint32_t sK0 = smem_u32(smem + L::OFF_K);
+      const uint32_t sV0 = smem_u32(smem + L::OFF_V);
+      const uint32_t sP0 = smem_u32(smem + L::OFF_P);
+      bool ok = n_steps == 0 || mbar_wait(bars.q_full, 0, wl, args.status, abort_flag);
+      for (int s = 0; ok && s <= n_steps; ++s) {
+        if (s < n_steps) {
+          const int st = s % NS;
+          if (!mbar_wait(bars.k_full + st, (s / NS) & 1, wl, args.status, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t d_s = tmem + (s & 1) * BK;
+          const uint32_t kbase = sK0 + st * L::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * (BM * 128) + off, 16, 1024);
+            const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * (BK * 128) + off, 16, 1024);
+            umma_ss(d_s, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bars.s_full + (s & 1));
+          umma_commit(bars.k_empty + st);
+        }
+        if (s >= 1) {
+          const int j = s - 1;
+          const int st = j % NS;
+          if (!mbar_wait(bars.p_full + (j & 1), (j >> 1) & 1, wl, args.status, abort_flag)) break;
+          if (!mbar_wait(bars.v_full + st, (j / NS) & 1, wl, args.status, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t pbase = sP0 + (j & 1) * L::P_BYTES;
+          const uint32_t vbase = sV0 + st * L::KV_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t a = smem_desc_sw128(pbase + kk * 32, 16, 1024);
+            const uint64_t b = smem_desc_sw128(vbase + kk * 2048, BK * 128, 1024);
+            umma_ss(tmem + 128, a, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bars.o_done + (j & 1));
+          umma_commit(bars.v_empty + st);
+        }
+      }
+      // drain: every UMMA this thread issued has completed before TMEM is released
+      umma_commit(bars.drain);
+      mbar_wait(bars.drain, 0, wl, args.status, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
+    const int row = tid;                       // tile row == TMEM lane
+    const int grow = tile * BM + row;          // token row
+    const int half = row >> 6;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m = -INFINITY;                       // running max (log2 units), possibly stale by < 8
+    float l = 0.f;
+    bool alive = true;
+    for (int s = 0; s < n_steps && alive; ++s) {
+      const int sb = s & 1;
+      if (!mbar_wait(bars.s_full + sb, (s >> 1) & 1, wl, args.status, abort_flag)) { alive = false; break; }
+      tc_fence_after();
+      const uint32_t e = sched[s / spb];
+      const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
+      const bool take = ((e >> 30) >> half) & 1u;
+      const int nvk = args.N_valid - key0;     // valid keys in this step (may exceed 64)
+      uint32_t r[64];
+      tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = (take && c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      const float m_new = fmaxf(m, mx);
+      const bool need = (m != -INFINITY) && (m_new > m + 8.0f);
+      if (m == -INFINITY) m = m_new;
+      if (__any_sync(0xffffffffu, need)) {
+        if (s >= 1 && !mbar_wait(bars.o_done + ((s - 1) & 1), ((s - 1) >> 1) & 1, wl, args.status, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = need ? ex2(m - m_new) : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + 128 + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+          tmem_st32(t_lane + 128 + c * 32, o);
+        }
+        tmem_wait_st();
+        if (need) {
+          l *= f;
+          m = m_new;
+        }
+      }
+      float sum = 0.f;
+      uint32_t pk[32];
+      const float mref = (m == -INFINITY) ? 0.f : m;   // a row that has seen no key yet: all p = 0
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2(x[2 * c] - mref);
+        const float p1 = ex2(x[2 * c + 1] - mref);
+        sum += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l += sum;
+      if (s >= 2 && !mbar_wait(bars.o_done + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) {
+        alive = false;
+        break;
+      }
+      // P row -> 128-byte-swizzled K-major tile: 16-byte chunk c of row `row`
+      // lands at chunk position (c ^ (row & 7)) of the row's 128-byte line.
+      uint8_t* prow = smem + L::OFF_P + sb * L::P_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars.p_full + sb);
+    }
+    // ---- epilogue: O / l  -> out, lse
+    bool ok_o = alive && n_steps > 0 && !*abort_flag;
+    if (ok_o) {
+      ok_o = mbar_wait(bars.o_done + ((n_steps - 1) & 1), ((n_steps - 1) >> 1) & 1, wl, args.status, abort_flag);
+      tc_fence_after();
+    }
+    const bool valid = grow < args.N_valid;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(args.out);
+    const long long obase = static_cast<long long>(bb) * args.ostride_b + static_cast<long long>(h) * args.ostride_h +
+                            static_cast<long long>(grow) * args.ostride_n;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      if (__all_sync(0xffffffffu, ok_o)) {
+        tmem_ld32(t_lane + 128 + c * 32, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (valid) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        uint4* dst = reinterpret_cast<uint4*>(outp + obase + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      }
+    }
+    if (args.lse && valid) {
+      const float v = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      args.lse[(static_cast<long long>(bb) * args.H + h) * args.N_valid + grow] = v;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                               const AttendArgs& a, cudaStream_t s) {
+  const int tiles = (a.N_valid + BM - 1) / BM;
+  dim3 grid(tiles, a.H, a.B);
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
+  if (a.nB > kMaxBlocks) return cudaErrorInvalidValue;
+  if (a.d == 128) {
+    const size_t smem = Layout<128>::bytes(a.nB);
+    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attend_bf16_kernel<128><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
+  } else {
+    const size_t smem = Layout<64>::bytes(a.nB);
+    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attend_bf16_kernel<64><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lbsa

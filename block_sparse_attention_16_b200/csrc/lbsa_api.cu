@@ -1,0 +1,428 @@
+// C ABI of liblbsa: argument validation, TMA tensor maps, blockset ownership,
+// status words, and dispatch to the kernels.  No torch types cross this
+// boundary: plain pointers, sizes and a cudaStream_t passed as void*.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "lbsa_device.cuh"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(e == cudaErrorMemoryAllocation ? LBSA_ERR_OOM : LBSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate_desc(const lbsa_qkv_desc* d) {
+  if (!d) return fail(LBSA_ERR_INVALID_ARG, "desc is NULL");
+  if (d->B < 1 || d->H < 1 || d->N_valid < 1)
+    return fail(LBSA_ERR_INVALID_ARG, "B, H and N_valid must be >= 1 (got %d, %d, %d)", d->B, d->H, d->N_valid);
+  if (d->dtype != LBSA_BF16 && d->dtype != LBSA_F32) return fail(LBSA_ERR_INVALID_ARG, "dtype %d unknown", d->dtype);
+  if (d->d != 64 && d->d != 128) return fail(LBSA_ERR_UNSUPPORTED, "head dim %d: only 64 and 128 are built", d->d);
+  const int es = d->dtype == LBSA_BF16 ? 2 : 4;
+  if (d->stride_n < d->d || d->stride_h < 1 || d->stride_b < 1)
+    return fail(LBSA_ERR_INVALID_ARG, "strides (%lld, %lld, %lld) smaller than a row", (long long)d->stride_b,
+                (long long)d->stride_h, (long long)d->stride_n);
+  if ((d->stride_n * es) % 16 || (d->stride_h * es) % 16 || (d->stride_b * es) % 16)
+    return fail(LBSA_ERR_INVALID_ARG, "byte strides must be multiples of 16");
+  if (static_cast<long long>(d->N_valid) >= (1ll << 31)) return fail(LBSA_ERR_INVALID_ARG, "N_valid too large");
+  return LBSA_OK;
+}
+
+int validate_ptr(const void* p, const char* name) {
+  if (!p) return fail(LBSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(LBSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return LBSA_OK;
+}
+
+int n_blocks(int n_valid, int block) { return (n_valid + block - 1) / block; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 [B, H, N_valid, d] as a 4D tensor map (d, N, H, B); box = 64 x box_rows,
+// 128-byte swizzle (each box row is one 128-byte swizzle line).
+int make_tmap(CUtensorMap* map, const void* ptr, const lbsa_qkv_desc* d, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d->d), static_cast<cuuint64_t>(d->N_valid),
+                        static_cast<cuuint64_t>(d->H), static_cast<cuuint64_t>(d->B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d->stride_n) * 2, static_cast<cuuint64_t>(d->stride_h) * 2,
+                           static_cast<cuuint64_t>(d->stride_b) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LBSA_OK;
+}
+
+// Per-device state: a status word for calls without a blockset and a
+// workspace that grows on demand (allocated outside the per-call path once it
+// is large enough).
+struct DeviceState {
+  int32_t* status = nullptr;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+};
+std::mutex g_mu;
+DeviceState g_dev[64];
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(LBSA_ERR_UNSUPPORTED, "device %d", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.status) {
+    e = cudaMalloc(&s.status, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status)");
+    e = cudaMemset(s.status, 0, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(status)");
+  }
+  *out = &s;
+  return LBSA_OK;
+}
+
+int workspace(DeviceState* s, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (s->ws_bytes < bytes) {
+    if (s->ws) {
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+      cudaFree(s->ws);
+      s->ws = nullptr;
+      s->ws_bytes = 0;
+    }
+    cudaError_t e = cudaMalloc(&s->ws, bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+    s->ws_bytes = bytes;
+  }
+  *out = s->ws;
+  return LBSA_OK;
+}
+
+long long wait_limit() { return lbsa::kDefaultWaitLimit; }
+
+int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStream_t s, lbsa_blockset** out) {
+  const size_t R = static_cast<size_t>(B) * H * nB;
+  const size_t cols_bytes = R * nB * sizeof(int32_t);
+  const size_t counts_bytes = ((R * sizeof(int32_t)) + 255) & ~size_t(255);
+  const size_t bytes = counts_bytes + cols_bytes + 256;
+  void* base = nullptr;
+  cudaError_t e = cudaMallocAsync(&base, bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(blockset)");
+  auto* bs = new lbsa_blockset;
+  bs->B = B;
+  bs->H = H;
+  bs->nB = nB;
+  bs->block = block;
+  bs->scope = scope;
+  bs->p = p;
+  bs->base = base;
+  bs->counts = static_cast<int32_t*>(base);
+  bs->cols = reinterpret_cast<int32_t*>(static_cast<char*>(base) + counts_bytes);
+  bs->status = reinterpret_cast<int32_t*>(static_cast<char*>(base) + counts_bytes + cols_bytes);
+  bs->stream = s;
+  cudaGetDevice(&bs->device);
+  e = cudaMemsetAsync(bs->status, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) {
+    cudaFreeAsync(base, s);
+    delete bs;
+    return cuda_fail(e, "cudaMemsetAsync");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int lbsa_version(void) { return 100; }
+
+const char* lbsa_last_error(void) { return g_err.c_str(); }
+
+int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t block, int32_t mode, float* scores,
+               float* lse, void* stream) {
+  int rc;
+  if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  if (mode != LBSA_SCORE_EXACT_MASS && mode != LBSA_SCORE_MEANPOOL) return fail(LBSA_ERR_INVALID_ARG, "mode %d", mode);
+  if (lse && mode != LBSA_SCORE_EXACT_MASS) return fail(LBSA_ERR_INVALID_ARG, "lse is only produced in exact mode");
+  const int nB = n_blocks(desc->N_valid, block);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != LBSA_OK) return rc;
+  cudaError_t e;
+  if (mode == LBSA_SCORE_EXACT_MASS) {
+    lbsa::ScoreArgs a{desc->B, desc->H, desc->N_valid, desc->d, block, nB, scores, lse, ds->status, wait_limit()};
+    if (desc->dtype == LBSA_BF16) {
+      CUtensorMap tq, tk;
+      if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
+      if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
+      e = lbsa::launch_score_exact_bf16(&tq, &tk, a, s);
+    } else {
+      e = lbsa::launch_score_exact_f32(static_cast<const float*>(q), static_cast<const float*>(k), *desc, a, s);
+    }
+  } else {
+    void* ws = nullptr;
+    if ((rc = workspace(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d), &ws)) != LBSA_OK) return rc;
+    e = lbsa::launch_meanpool(q, k, *desc, block, nB, scores, ws, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_score launch");
+  return LBSA_OK;
+}
+
+int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p, int32_t scope,
+                lbsa_blockset** out, void* stream) {
+  int rc;
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if (B < 1 || H < 1 || nB < 1) return fail(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
+  if (scope != LBSA_SCOPE_ROW && scope != LBSA_SCOPE_HEAD) return fail(LBSA_ERR_INVALID_ARG, "scope %d", scope);
+  if (scope == LBSA_SCOPE_ROW && nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "row scope is built for nB <= 1024");
+  if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "nB %d > 4096", nB);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  if ((rc = new_blockset(B, H, nB, block, scope, p, s, &bs)) != LBSA_OK) return rc;
+  cudaError_t e;
+  if (scope == LBSA_SCOPE_ROW) {
+    e = lbsa::launch_select_row(scores, B * H * nB, nB, p, bs, s);
+  } else {
+    DeviceState* ds = nullptr;
+    void* ws = nullptr;
+    if ((rc = device_state(&ds)) != LBSA_OK || (rc = workspace(ds, lbsa::select_head_workspace_bytes(B, H, nB), &ws)) != LBSA_OK) {
+      lbsa_free(bs);
+      return rc;
+    }
+    e = lbsa::launch_select_head(scores, B, H, nB, p, bs, ws, s);
+  }
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_select launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
+int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, const lbsa_blockset* bs,
+                void* out, float* lse, void* stream) {
+  int rc;
+  if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(v, "v")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(out, "out")) != LBSA_OK) return rc;
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (bs->B != desc->B || bs->H != desc->H || bs->nB != n_blocks(desc->N_valid, bs->block))
+    return fail(LBSA_ERR_INVALID_ARG, "blockset (B=%d, H=%d, nB=%d, block=%d) does not match q (B=%d, H=%d, N=%d)",
+                bs->B, bs->H, bs->nB, bs->block, desc->B, desc->H, desc->N_valid);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != bs->device) return fail(LBSA_ERR_INVALID_ARG, "blockset lives on device %d, current is %d", bs->device, dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa::AttendArgs a{desc->B, desc->H, desc->N_valid, desc->d, bs->block, bs->nB, bs->counts, bs->cols, bs->status,
+                     out, desc->stride_b, desc->stride_h, desc->stride_n, lse, wait_limit()};
+  cudaError_t e;
+  if (desc->dtype == LBSA_BF16) {
+    CUtensorMap tq, tk, tv;
+    if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
+    if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
+    if ((rc = make_tmap(&tv, v, desc, 64)) != LBSA_OK) return rc;
+    e = lbsa::launch_attend_bf16(&tq, &tk, &tv, a, s);
+  } else {
+    e = lbsa::launch_attend_f32(static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+                                *desc, a, s);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_attend launch");
+  return LBSA_OK;
+}
+
+void lbsa_free(lbsa_blockset* bs) {
+  if (!bs) return;
+  if (bs->base) cudaFreeAsync(bs->base, bs->stream);
+  delete bs;
+}
+
+int lbsa_blockset_info(const lbsa_blockset* bs, int32_t* B, int32_t* H, int32_t* nB, int32_t* block, int32_t* scope) {
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (B) *B = bs->B;
+  if (H) *H = bs->H;
+  if (nB) *nB = bs->nB;
+  if (block) *block = bs->block;
+  if (scope) *scope = bs->scope;
+  return LBSA_OK;
+}
+
+int lbsa_blockset_views(const lbsa_blockset* bs, const int32_t** counts, const int32_t** cols) {
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (counts) *counts = bs->counts;
+  if (cols) *cols = bs->cols;
+  return LBSA_OK;
+}
+
+int lbsa_blockset_export(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col, int64_t* nnz, void* stream) {
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (!row_ptr || !col || !nnz) return fail(LBSA_ERR_INVALID_ARG, "row_ptr, col and nnz must be non-NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* d_nnz = row_ptr + static_cast<long long>(bs->B) * bs->H * bs->nB;   // row_ptr[R] holds the total
+  cudaError_t e = lbsa::launch_export_csr(bs, row_ptr, col, d_nnz, s);
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_blockset_export launch");
+  int32_t h = 0;
+  e = cudaMemcpyAsync(&h, d_nnz, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_blockset_export copy");
+  *nnz = h;
+  return LBSA_OK;
+}
+
+int lbsa_blockset_from_csr(const int32_t* row_ptr, const int32_t* col, int32_t B, int32_t H, int32_t nB, int32_t block,
+                           lbsa_blockset** out, void* stream) {
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!row_ptr || !col) return fail(LBSA_ERR_INVALID_ARG, "row_ptr and col must be non-NULL");
+  if (B < 1 || H < 1 || nB < 1 || nB > 4096) return fail(LBSA_ERR_INVALID_ARG, "bad B/H/nB");
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d", block);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  int rc = new_blockset(B, H, nB, block, LBSA_SCOPE_ROW, -1.0, s, &bs);
+  if (rc != LBSA_OK) return rc;
+  cudaError_t e = lbsa::launch_from_csr(row_ptr, col, bs, s);
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_blockset_from_csr launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
+int lbsa_get_status(const lbsa_blockset* bs, int32_t* device_status, int32_t clear, void* stream) {
+  if (!bs || !device_status) return fail(LBSA_ERR_INVALID_ARG, "NULL argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(device_status, bs->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(bs->status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_get_status");
+  return LBSA_OK;
+}
+
+int lbsa_device_status(int32_t* device_status, int32_t clear, void* stream) {
+  if (!device_status) return fail(LBSA_ERR_INVALID_ARG, "NULL argument");
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LBSA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(device_status, ds->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(ds->status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_device_status");
+  return LBSA_OK;
+}
+
+int lbsa_partition_perm(int32_t T, int32_t Hg, int32_t Wg, int32_t kind, int32_t tt, int32_t th, int32_t tw,
+                        int32_t* perm, int32_t on_device, void* stream) {
+  if (!perm) return fail(LBSA_ERR_INVALID_ARG, "perm is NULL");
+  if (T < 1 || Hg < 1 || Wg < 1) return fail(LBSA_ERR_INVALID_ARG, "grid must be >= 1 in every axis");
+  if (static_cast<long long>(T) * Hg * Wg >= (1ll << 31)) return fail(LBSA_ERR_INVALID_ARG, "grid too large");
+  if (kind < LBSA_PART_RASTER || kind > LBSA_PART_3D) return fail(LBSA_ERR_INVALID_ARG, "partition kind %d", kind);
+  if ((kind == LBSA_PART_2D && (th < 1 || tw < 1)) || (kind == LBSA_PART_3D && (tt < 1 || th < 1 || tw < 1)))
+    return fail(LBSA_ERR_INVALID_ARG, "tile sizes must be >= 1");
+  if (!on_device) {
+    lbsa::partition_perm_host(T, Hg, Wg, kind, tt, th, tw, perm);
+    return LBSA_OK;
+  }
+  cudaError_t e = lbsa::launch_partition_perm(T, Hg, Wg, kind, tt, th, tw, perm, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_partition_perm launch");
+  return LBSA_OK;
+}
+
+int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const int32_t* perm, const lbsa_qkv_desc* desc,
+                 int32_t inverse, void* stream) {
+  int rc;
+  if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
+  if (!xs || !ys || count < 1 || count > 3) return fail(LBSA_ERR_INVALID_ARG, "need 1..3 tensors");
+  if (!perm) return fail(LBSA_ERR_INVALID_ARG, "perm is NULL");
+  for (int t = 0; t < count; ++t) {
+    if ((rc = validate_ptr(xs[t], "x")) != LBSA_OK) return rc;
+    if ((rc = validate_ptr(ys[t], "y")) != LBSA_OK) return rc;
+    if (xs[t] == ys[t]) return fail(LBSA_ERR_INVALID_ARG, "x and y may not alias");
+  }
+  cudaError_t e = lbsa::launch_permute(xs, ys, count, perm, *desc, inverse, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_permute launch");
+  return LBSA_OK;
+}
+
+int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream) {
+  if (!device_out) return fail(LBSA_ERR_INVALID_ARG, "device_out is NULL");
+  if (iters < 1 || iters > (1ll << 30)) return fail(LBSA_ERR_INVALID_ARG, "iters out of range");
+  cudaError_t e = lbsa::launch_selftest_wait(iters, device_out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_selftest_wait launch");
+  return LBSA_OK;
+}
+
+}  // extern "C"
+
+namespace lbsa {
+namespace {
+// One thread waits on an mbarrier that nothing ever completes.
+__global__ void selftest_wait_kernel(long long iters, int32_t* out) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  __shared__ int32_t st;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    st = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = mbar_wait(&bar, 0, iters, &st, &abort_flag);
+    *out = ok ? LBSA_OK : st;
+  }
+}
+}  // namespace
+
+cudaError_t launch_selftest_wait(long long iters, int32_t* out, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(iters, out);
+  return cudaGetLastError();
+}
+}  // namespace lbsa

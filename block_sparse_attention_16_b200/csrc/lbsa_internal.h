@@ -1,0 +1,83 @@
+// Internal declarations shared by the C ABI layer and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/lbsa.h"
+
+// Library-owned selection result.  Row r = (b*H + h)*nB + i owns the slot
+// cols[r*nB .. r*nB + nB); counts[r] entries of it are valid, ascending.
+struct lbsa_blockset {
+  int32_t B, H, nB, block, scope;
+  double p;
+  int32_t* counts;      // device [R]
+  int32_t* cols;        // device [R * nB]
+  int32_t* status;      // device [1]
+  void* base;           // single stream-ordered allocation holding the three arrays
+  cudaStream_t stream;  // stream it was created on (freed on it)
+  int device;
+};
+
+namespace lbsa {
+
+constexpr long long kDefaultWaitLimit = 1ll << 20;   // mbarrier polls before a wait gives up (~1 s)
+
+struct AttendArgs {
+  int B, H, N_valid, d, block, nB;
+  const int32_t* counts;
+  const int32_t* cols;
+  int32_t* status;
+  void* out;
+  int64_t ostride_b, ostride_h, ostride_n;   // elements
+  float* lse;
+  long long wait_limit;
+};
+
+struct ScoreArgs {
+  int B, H, N_valid, d, block, nB;
+  float* scores;
+  float* lse;
+  int32_t* status;
+  long long wait_limit;
+};
+
+// bf16 tcgen05 kernels (attend_tc.cu, score_tc.cu)
+cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                               const AttendArgs& a, cudaStream_t s);
+cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
+                                    cudaStream_t s);
+
+// fp32 SIMT kernels (simt_f32.cu)
+cudaError_t launch_attend_f32(const float* q, const float* k, const float* v, const lbsa_qkv_desc& d,
+                              const AttendArgs& a, cudaStream_t s);
+cudaError_t launch_score_exact_f32(const float* q, const float* k, const lbsa_qkv_desc& d,
+                                   const ScoreArgs& a, cudaStream_t s);
+
+// block-mean proxy (meanpool.cu); workspace holds 2*B*H*nB*d floats + partials
+size_t meanpool_workspace_bytes(int B, int H, int nB, int d);
+cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB,
+                            float* scores, void* workspace, cudaStream_t s);
+
+// selection (select.cu)
+cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,
+                              cudaStream_t s);
+size_t select_head_workspace_bytes(int B, int H, int nB);
+cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs,
+                               void* workspace, cudaStream_t s);
+cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col,
+                              int32_t* nnz_dev, cudaStream_t s);
+cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blockset* bs,
+                            cudaStream_t s);
+
+// permutation (permute.cu)
+void partition_perm_host(int T, int Hg, int Wg, int kind, int tt, int th, int tw, int32_t* perm);
+cudaError_t launch_partition_perm(int T, int Hg, int Wg, int kind, int tt, int th, int tw,
+                                  int32_t* perm, cudaStream_t s);
+cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, const int32_t* perm,
+                           const lbsa_qkv_desc& d, int inverse, cudaStream_t s);
+
+cudaError_t launch_selftest_wait(long long iters, int32_t* out, cudaStream_t s);
+
+}  // namespace lbsa

@@ -1,0 +1,204 @@
+// Block-mean proxy scores (VMoBA review on pith.science, arXiv 2506.23858,
+// "What carries the argument": every key block is represented by its mean key
+// and queries score these block means).  Block-granular reading: the query
+// side is pooled the same way, and the similarities of one head are
+// normalised by a softmax over all of its query-block x key-block pairs:
+//   qbar_i = mean_{r in I_i} q_r,  kbar_j = mean_{c in J_j} k_c   (fp32)
+//   s_ij = qbar_i . kbar_j / sqrt(d)
+//   score[b,h,i,j] = exp(s_ij - M) / sum_{i',j'} exp(s_i'j' - M),  M = max s
+// Three kernels: block means (reads Q and K once, 16-byte loads), the 64x64
+// tiles of s with per-tile (max, sum of exp), and the normalisation.
+#include "lbsa_device.cuh"
+
+#include <cuda_bf16.h>
+
+namespace lbsa {
+namespace {
+
+constexpr int kTile = 64;
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// grid (nB, H, B), 256 threads: thread = (row group g, 8-column vector v).
+template <typename T, int D>
+__global__ void block_mean_kernel(const T* __restrict__ q, const T* __restrict__ k, lbsa_qkv_desc desc, int block,
+                                  int nB, float* __restrict__ qbar, float* __restrict__ kbar) {
+  constexpr int V = D / 8;               // vectors per row
+  constexpr int G = 256 / V;             // row groups
+  __shared__ float red[2][G][D];
+  const int i = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+  const int v = threadIdx.x % V, g = threadIdx.x / V;
+  const int r0 = i * block, r1 = min(r0 + block, desc.N_valid);
+  const long long base = bb * desc.stride_b + h * desc.stride_h;
+  float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int r = r0 + g; r < r1; r += G) {
+    float f[8];
+    load8(q + base + r * desc.stride_n + v * 8, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) aq[e] += f[e];
+    load8(k + base + r * desc.stride_n + v * 8, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ak[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    red[0][g][v * 8 + e] = aq[e];
+    red[1][g][v * 8 + e] = ak[e];
+  }
+  __syncthreads();
+  const float inv = 1.0f / static_cast<float>(r1 - r0);
+  const long long o = ((static_cast<long long>(bb) * desc.H + h) * nB + i) * D;
+  for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
+    const int which = c / D, col = c % D;
+    float s = 0.f;
+    for (int gg = 0; gg < G; ++gg) s += red[which][gg][col];
+    (which ? kbar : qbar)[o + col] = s * inv;
+  }
+}
+
+// grid (nT, nT, B*H) with nT = ceil(nB/64); 256 threads, each a 4x4 patch of s.
+template <int D>
+__global__ void logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nB, float scale,
+                              float* __restrict__ scores, float2* __restrict__ part) {
+  constexpr int KC = 32;                 // columns of d staged per round
+  __shared__ float sq[kTile][KC + 1];
+  __shared__ float sk[kTile][KC + 1];
+  __shared__ float red_m[256], red_s[256];
+  const int ti = blockIdx.y, tj = blockIdx.x, g = blockIdx.z;
+  const int nT = gridDim.x;
+  const float* qb = qbar + static_cast<long long>(g) * nB * D;
+  const float* kb = kbar + static_cast<long long>(g) * nB * D;
+  const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
+  float acc[4][4] = {};
+  for (int c0 = 0; c0 < D; c0 += KC) {
+    for (int e = threadIdx.x; e < kTile * KC; e += 256) {
+      const int r = e / KC, c = e % KC;
+      const int qi = ti * kTile + r, kj = tj * kTile + r;
+      sq[r][c] = (qi < nB) ? qb[static_cast<long long>(qi) * D + c0 + c] : 0.f;
+      sk[r][c] = (kj < nB) ? kb[static_cast<long long>(kj) * D + c0 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int c = 0; c < KC; ++c) {
+      float a[4], b[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] = sq[tr + u][c];
+        b[u] = sk[tc + u][c];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+    }
+    __syncthreads();
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int qi = ti * kTile + tr + u, kj = tj * kTile + tc + w;
+      acc[u][w] *= scale;
+      if (qi < nB && kj < nB) {
+        scores[(static_cast<long long>(g) * nB + qi) * nB + kj] = acc[u][w];
+        mx = fmaxf(mx, acc[u][w]);
+      }
+    }
+  red_m[threadIdx.x] = mx;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red_m[threadIdx.x] = fmaxf(red_m[threadIdx.x], red_m[threadIdx.x + o]);
+    __syncthreads();
+  }
+  const float tm = red_m[0];
+  float sm = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int qi = ti * kTile + tr + u, kj = tj * kTile + tc + w;
+      if (qi < nB && kj < nB) sm += expf(acc[u][w] - tm);
+    }
+  red_s[threadIdx.x] = sm;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red_s[threadIdx.x] += red_s[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[(static_cast<long long>(g) * nT + ti) * nT + tj] = make_float2(tm, red_s[0]);
+}
+
+// grid (chunks, B*H), 256 threads: combine the head's tile partials (fixed
+// order), then normalise a chunk of the head's scores in place.
+__global__ void normalize_kernel(float* __restrict__ scores, const float2* __restrict__ part, int nB, int nT) {
+  __shared__ float sM, sZ;
+  const int g = blockIdx.y;
+  const float2* pp = part + static_cast<long long>(g) * nT * nT;
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int t = 0; t < nT * nT; ++t) M = fmaxf(M, pp[t].x);
+    float Z = 0.f;
+    for (int t = 0; t < nT * nT; ++t) Z += pp[t].y * expf(pp[t].x - M);
+    sM = M;
+    sZ = Z;
+  }
+  __syncthreads();
+  const float M = sM, invZ = 1.0f / sZ;
+  const long long n = static_cast<long long>(nB) * nB;
+  float* s = scores + static_cast<long long>(g) * n;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    s[i] = expf(s[i] - M) * invZ;
+}
+
+template <int D>
+cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, float* scores, void* ws,
+                cudaStream_t s) {
+  const long long G = static_cast<long long>(d.B) * d.H;
+  float* qbar = static_cast<float*>(ws);
+  float* kbar = qbar + G * nB * D;
+  float2* part = reinterpret_cast<float2*>(kbar + G * nB * D);
+  const int nT = (nB + kTile - 1) / kTile;
+  if (d.dtype == LBSA_BF16)
+    block_mean_kernel<__nv_bfloat16, D><<<dim3(nB, d.H, d.B), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), d, block, nB, qbar, kbar);
+  else
+    block_mean_kernel<float, D><<<dim3(nB, d.H, d.B), 256, 0, s>>>(static_cast<const float*>(q),
+                                                                    static_cast<const float*>(k), d, block, nB,
+                                                                    qbar, kbar);
+  logits_kernel<D><<<dim3(nT, nT, static_cast<unsigned>(G)), 256, 0, s>>>(
+      qbar, kbar, nB, static_cast<float>(1.0 / std::sqrt(static_cast<double>(D))), scores, part);
+  const int chunks = static_cast<int>(std::min<long long>(64, (static_cast<long long>(nB) * nB + 2047) / 2048));
+  normalize_kernel<<<dim3(chunks, static_cast<unsigned>(G)), 256, 0, s>>>(scores, part, nB, nT);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t meanpool_workspace_bytes(int B, int H, int nB, int d) {
+  const size_t G = static_cast<size_t>(B) * H;
+  const size_t nT = (nB + kTile - 1) / kTile;
+  return 2 * G * nB * d * sizeof(float) + G * nT * nT * sizeof(float2) + 256;
+}
+
+cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, float* scores,
+                            void* ws, cudaStream_t s) {
+  return d.d == 128 ? run<128>(q, k, d, block, nB, scores, ws, s) : run<64>(q, k, d, block, nB, scores, ws, s);
+}
+
+}  // namespace lbsa

@@ -1,0 +1,114 @@
+// Token orders for VMoBA's 1D / 2D / 3D block partitions (pith.science review
+// of arXiv 2506.23858: layer-wise cyclic 1D-2D-3D partition) and the row
+// gather / scatter that puts Q, K, V into block order and O back.
+//
+// slot_of(t, h, w) gives the blocked position of the raster token (t, h, w) in
+// closed form: tiles are visited in raster tile order and tokens in raster
+// order inside a tile, with edge tiles truncated, so every tile before the
+// token's tile in its tile-row / tile-slab is full-sized along the axes that
+// are already passed.
+#include "lbsa_device.cuh"
+
+namespace lbsa {
+namespace {
+
+__host__ __device__ inline long long slot_of(int t, int h, int w, int T, int Hg, int Wg, int kind, int tt, int th,
+                                             int tw) {
+  switch (kind) {
+    case LBSA_PART_1D:
+      return (static_cast<long long>(h) * Wg + w) * T + t;
+    case LBSA_PART_2D: {
+      const int a = h / th, c = w / tw;
+      const int sh = min(th, Hg - a * th), sw = min(tw, Wg - c * tw);
+      const long long frame = static_cast<long long>(t) * Hg * Wg;
+      return frame + static_cast<long long>(a) * th * Wg + static_cast<long long>(sh) * c * tw +
+             static_cast<long long>(h - a * th) * sw + (w - c * tw);
+    }
+    case LBSA_PART_3D: {
+      const int at = t / tt, a = h / th, c = w / tw;
+      const int st = min(tt, T - at * tt), sh = min(th, Hg - a * th), sw = min(tw, Wg - c * tw);
+      return static_cast<long long>(at) * tt * Hg * Wg + static_cast<long long>(st) * a * th * Wg +
+             static_cast<long long>(st) * sh * c * tw +
+             (static_cast<long long>(t - at * tt) * sh + (h - a * th)) * sw + (w - c * tw);
+    }
+    default:
+      return (static_cast<long long>(t) * Hg + h) * Wg + w;
+  }
+}
+
+__global__ void partition_perm_kernel(int T, int Hg, int Wg, int kind, int tt, int th, int tw, int32_t* perm) {
+  const long long n = static_cast<long long>(T) * Hg * Wg;
+  for (long long tok = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; tok < n;
+       tok += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int w = static_cast<int>(tok % Wg);
+    const int h = static_cast<int>((tok / Wg) % Hg);
+    const int t = static_cast<int>(tok / (static_cast<long long>(Wg) * Hg));
+    perm[slot_of(t, h, w, T, Hg, Wg, kind, tt, th, tw)] = static_cast<int32_t>(tok);
+  }
+}
+
+// One thread per 16-byte vector of a row; vec_per_row = d * esize / 16 and the
+// strides are in 16-byte vectors.  Up to three tensors share perm.
+struct PtrPack {
+  const uint4* x[3];
+  uint4* y[3];
+};
+
+__global__ void permute_kernel_packed(PtrPack pk, int count, const int32_t* __restrict__ perm, int B, int H, int N,
+                                      int vec_per_row, long long sb, long long sh, long long sn, int inverse) {
+  const long long per_t = static_cast<long long>(B) * H * N * vec_per_row;
+  const long long total = per_t * count;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / per_t);
+    long long r = i - t * per_t;
+    const int v = static_cast<int>(r % vec_per_row);
+    r /= vec_per_row;
+    const int slot = static_cast<int>(r % N);
+    r /= N;
+    const int h = static_cast<int>(r % H);
+    const int b = static_cast<int>(r / H);
+    const int src = __ldg(perm + slot);
+    const long long base = b * sb + h * sh;
+    const uint4* x = pk.x[t];
+    uint4* y = pk.y[t];
+    if (!inverse) y[base + slot * sn + v] = __ldg(x + base + src * sn + v);
+    else y[base + src * sn + v] = __ldg(x + base + slot * sn + v);
+  }
+}
+
+}  // namespace
+
+void partition_perm_host(int T, int Hg, int Wg, int kind, int tt, int th, int tw, int32_t* perm) {
+  for (int t = 0; t < T; ++t)
+    for (int h = 0; h < Hg; ++h)
+      for (int w = 0; w < Wg; ++w)
+        perm[slot_of(t, h, w, T, Hg, Wg, kind, tt, th, tw)] = (t * Hg + h) * Wg + w;
+}
+
+cudaError_t launch_partition_perm(int T, int Hg, int Wg, int kind, int tt, int th, int tw, int32_t* perm,
+                                  cudaStream_t s) {
+  const long long n = static_cast<long long>(T) * Hg * Wg;
+  const int blocks = static_cast<int>(std::min<long long>((n + 255) / 256, 148 * 8));
+  partition_perm_kernel<<<blocks, 256, 0, s>>>(T, Hg, Wg, kind, tt, th, tw, perm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, const int32_t* perm,
+                           const lbsa_qkv_desc& d, int inverse, cudaStream_t s) {
+  const int esize = d.dtype == LBSA_BF16 ? 2 : 4;
+  const int vec_per_row = d.d * esize / 16;
+  const long long k = 16 / esize;   // elements per vector
+  PtrPack pk{};
+  for (int t = 0; t < count; ++t) {
+    pk.x[t] = static_cast<const uint4*>(xs[t]);
+    pk.y[t] = static_cast<uint4*>(ys[t]);
+  }
+  const long long total = static_cast<long long>(count) * d.B * d.H * d.N_valid * vec_per_row;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
+  permute_kernel_packed<<<blocks, 256, 0, s>>>(pk, count, perm, d.B, d.H, d.N_valid, vec_per_row, d.stride_b / k,
+                                               d.stride_h / k, d.stride_n / k, inverse);
+  return cudaGetLastError();
+}
+
+}  // namespace lbsa

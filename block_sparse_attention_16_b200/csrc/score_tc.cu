@@ -1,0 +1,251 @@
+// Exact block attention mass on sm_100a tensor cores (bf16 in, fp32 out).
+//
+// LoSA (abstract, scholarbro.com author page of C. Sun) measures the exact
+// block attention masses at one dense step.  Reading used for how the rows of a
+// query block combine: the mean over the block's valid rows, so
+//   mass[b,h,i,j] = (1/|I_i|) sum_{r in I_i} sum_{c in J_j} softmax_c(q_r.k_c/sqrt(d)).
+//
+// One CTA owns a 128-row query tile and sweeps the whole key sequence twice in
+// 64-key steps: sweep 1 builds each row's log-sum-exp (online max / sum),
+// sweep 2 recomputes S = Q K^T, forms p = exp(s - lse) and sums it per row
+// over each 64-key chunk; warp shuffles reduce the chunk sums over the rows of
+// a warp, and the per-warp partials are combined in a fixed order at the end
+// (deterministic).  The row log-sum-exp stays in registers between sweeps, so
+// the kernel needs no memory beyond its inputs and outputs.
+//
+// Warp roles (192 threads, two CTAs per SM): warps 0-3 softmax (thread t = tile
+// row t = TMEM lane t), warp 4 TMA producer (Q once, K 64-key tiles through a
+// ring), warp 5 UMMA issuer (S = Q K^T, M=128, N=64, K=d, double-buffered in
+// TMEM columns [0,64) and [64,128)).
+#include "lbsa_device.cuh"
+
+namespace lbsa {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NS = 3;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 128;
+
+template <int D>
+struct Layout {
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int K_BYTES = BK * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_BAR = OFF_K + NS * K_BYTES;
+  // q_full, k_full[NS], k_empty[NS], s_full[2], s_free[2], drain
+  static constexpr int NBAR = 1 + 2 * NS + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_PART = OFF_MISC + 16;
+  static size_t bytes(int n_chunks) { return OFF_PART + static_cast<size_t>(4) * n_chunks * 4 + 1024; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                        const ScoreArgs args, float scale_log2) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
+  const int N = args.N_valid;
+  const int n_chunks = (N + BK - 1) / BK;
+  const int n_steps = 2 * n_chunks;
+  const long long wl = args.wait_limit;
+  if (*reinterpret_cast<volatile int32_t*>(args.status) == LBSA_ERR_TIMEOUT) return;
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bar;
+  uint64_t* k_full = bar + 1;
+  uint64_t* k_empty = bar + 1 + NS;
+  uint64_t* s_full = bar + 1 + 2 * NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* drain = s_free + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  float* part = reinterpret_cast<float*>(smem + L::OFF_PART);   // [4][n_chunks]
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(s_free + i, 128);
+    }
+    mbar_init(drain, 1);
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(misc, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tmap_q);
+      prefetch_tmap(&tmap_k);
+      uint8_t* sQ = smem + L::OFF_Q;
+      mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+      for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, q_full, c * 64, tile * BM, h, bb);
+      int issued = 0;
+      for (int s = 0; s < n_steps; ++s) {
+        const int st = s % NS;
+        if (s >= NS && !mbar_wait(k_empty + st, ((s / NS) & 1) ^ 1, wl, args.status, abort_flag)) break;
+        const int key0 = (s % n_chunks) * BK;
+        uint8_t* sK = smem + L::OFF_K + st * L::K_BYTES;
+        mbar_arrive_expect_tx(k_full + st, L::K_BYTES);
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, key0, h, bb);
+        issued = s + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(q_full, 0, wl, args.status, nullptr);
+        for (int s = (issued > NS ? issued - NS : 0); s < issued; ++s)
+          mbar_wait(k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BK, 0);
+      const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+      const uint32_t sK0 = smem_u32(smem + L::OFF_K);
+      bool ok = mbar_wait(q_full, 0, wl, args.status, abort_flag);
+      for (int s = 0; ok && s < n_steps; ++s) {
+        const int st = s % NS;
+        const int sb = s & 1;
+        if (!mbar_wait(k_full + st, (s / NS) & 1, wl, args.status, abort_flag)) break;
+        if (s >= 2 && !mbar_wait(s_free + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t kbase = sK0 + st * L::K_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * (BM * 128) + off, 16, 1024);
+          const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * (BK * 128) + off, 16, 1024);
+          umma_ss(tmem + sb * BK, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full + sb);
+        umma_commit(k_empty + st);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, wl, args.status, nullptr);
+    }
+  } else {
+    const int row = tid;
+    const int grow = tile * BM + row;
+    const bool valid_row = grow < N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m = -INFINITY, l = 0.f, lse2 = 0.f;
+    for (int s = 0; s < n_steps; ++s) {
+      const int sb = s & 1;
+      if (!mbar_wait(s_full + sb, (s >> 1) & 1, wl, args.status, abort_flag)) break;
+      tc_fence_after();
+      uint32_t r[64];
+      tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_free + sb);
+      const int chunk = s % n_chunks;
+      const int nvk = N - chunk * BK;
+      if (s < n_chunks) {
+        float x[64];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] = (c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        const float m_new = fmaxf(m, mx);
+        float acc = (m == -INFINITY) ? 0.f : l * ex2(m - m_new);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc += ex2(x[c] - m_new);
+        l = acc;
+        m = m_new;
+        if (s == n_chunks - 1) lse2 = m + __log2f(l);
+      } else {
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          rs += (c < nvk) ? ex2(__uint_as_float(r[c]) * scale_log2 - lse2) : 0.f;
+        if (!valid_row) rs = 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+        if (lane == 0) part[warp * n_chunks + chunk] = rs;
+      }
+    }
+    named_bar_sync(1, 128);
+    if (!*abort_flag) {
+      const int nB = args.nB;
+      const long long hrow = (static_cast<long long>(bb) * args.H + h) * nB;
+      if (args.block == 64) {
+        for (int o = tid; o < 2 * nB; o += 128) {
+          const int half = o / nB, kb = o % nB;
+          const int qb = 2 * tile + half;
+          if (qb >= nB) continue;
+          const int rv = min(64, N - qb * 64);
+          const float v = (part[(2 * half) * n_chunks + kb] + part[(2 * half + 1) * n_chunks + kb]) / static_cast<float>(rv);
+          args.scores[(hrow + qb) * nB + kb] = v;
+        }
+      } else {
+        const int qb = tile;
+        const int rv = min(128, N - qb * 128);
+        for (int kb = tid; kb < nB; kb += 128) {
+          float v = 0.f;
+          for (int half = 0; half < 2; ++half) {
+            const int c = 2 * kb + half;
+            if (c < n_chunks)
+              v += (part[c] + part[n_chunks + c]) + (part[2 * n_chunks + c] + part[3 * n_chunks + c]);
+          }
+          args.scores[(hrow + qb) * nB + kb] = v / static_cast<float>(rv);
+        }
+      }
+      if (args.lse && valid_row)
+        args.lse[(static_cast<long long>(bb) * args.H + h) * N + grow] = lse2 * 0.69314718055994531f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
+                                    cudaStream_t s) {
+  const int tiles = (a.N_valid + BM - 1) / BM;
+  const int n_chunks = (a.N_valid + BK - 1) / BK;
+  dim3 grid(tiles, a.H, a.B);
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
+  if (a.d == 128) {
+    const size_t smem = Layout<128>::bytes(n_chunks);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(score_exact_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    score_exact_bf16_kernel<128><<<grid, kThreads, smem, s>>>(*tq, *tk, a, scale_log2);
+  } else {
+    const size_t smem = Layout<64>::bytes(n_chunks);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(score_exact_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    score_exact_bf16_kernel<64><<<grid, kThreads, smem, s>>>(*tq, *tk, a, scale_log2);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lbsa

@@ -1,0 +1,476 @@
+// Mass-threshold block selection (LoSA abstract: per head and query block, the
+// smallest key/value block set whose retained mass meets the threshold; VMoBA
+// review on pith.science, circularity check: the smallest k' whose cumulative
+// normalized similarity reaches tau, with VMoBA's global selection over all
+// block pairs of a head, where query rows may come out empty).
+//
+// The cumulative sum is exact so that the kept set does not depend on the
+// order of a parallel reduction:
+//   w = floor(x * 2^32)  (x fp32 in [0, 2): w < 2^33, computed from the bits)
+//   W = sum w,  P = round_half_even(p * 2^24),  T = ceil(P * W / 2^24)
+//   order by x descending, then flat index ascending; keep the shortest
+//   prefix whose sum of w reaches T (at least one element); p >= 1 keeps all.
+// Instead of sorting, both scopes search for the threshold value tb: the
+// largest bit pattern whose "weight at or above" S(tb) = sum_{bits >= tb} w
+// still reaches T.  Every element above tb is kept; of the elements equal to
+// tb (all of weight w(tb)), the ceil((T - S(tb+1)) / w(tb)) with the lowest
+// flat indices are kept.  This is exactly the sorted-prefix rule.
+#include "lbsa_device.cuh"
+
+namespace lbsa {
+namespace {
+
+constexpr uint32_t kInvalidBits = 0x40000000u;    // bits >= this: NaN, inf, negative, or >= 2.0
+
+// floor(x * 2^32) for a valid fp32 bit pattern (0 <= x < 2), in integers.
+__device__ __forceinline__ uint64_t fixed_weight(uint32_t bits) {
+  const uint32_t e = bits >> 23;
+  if (e == 0) return 0;                       // zero / subnormal: x * 2^32 < 1
+  const uint64_t M = (bits & 0x7FFFFFu) | 0x800000u;
+  if (e >= 118) return M << (e - 118);
+  const uint32_t sh = 118 - e;
+  return sh >= 24 ? 0 : (M >> sh);
+}
+
+__device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint64_t threshold_T(uint64_t W, uint32_t Pfix) {
+  const unsigned __int128 num = static_cast<unsigned __int128>(W) * Pfix + ((1u << 24) - 1);
+  return static_cast<uint64_t>(num >> 24);
+}
+
+// ---------------------------------------------------------------- row scope
+// One warp per row of nB scores; lane l holds elements l, l+32, ...
+template <int EPL>
+__global__ void select_row_kernel(const float* __restrict__ scores, int R, int nB, uint32_t Pfix, int keep_all,
+                                  int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+                                  int32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
+  int32_t* out = cols + row * nB;
+  uint32_t bits[EPL];
+  uint64_t w[EPL];
+  bool bad = false;
+  uint64_t wsum = 0;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int idx = e * 32 + lane;
+    const uint32_t b = (idx < nB) ? __ldg(x + idx) : 0u;
+    bad |= (idx < nB) && (b >= kInvalidBits);
+    bits[e] = b;
+    w[e] = (idx < nB && b < kInvalidBits) ? fixed_weight(b) : 0;
+    wsum += w[e];
+  }
+  const bool any_bad = __any_sync(0xffffffffu, bad);
+  if (any_bad || keep_all) {
+    if (any_bad && lane == 0) raise_status(status, LBSA_ERR_INVALID_SCORES);
+    for (int idx = lane; idx < nB; idx += 32) out[idx] = idx;
+    if (lane == 0) counts[row] = nB;
+    return;
+  }
+  const uint64_t W = warp_sum_u64(wsum);
+  const uint64_t T = threshold_T(W, Pfix);
+  uint32_t tb;
+  uint32_t need;
+  if (T == 0) {
+    // nothing to reach: keep one block, the highest score with the lowest index
+    uint32_t mb = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e)
+      if (e * 32 + lane < nB) mb = max(mb, bits[e]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    tb = mb;
+    need = 1;
+  } else {
+    uint32_t lo = 0, hi = kInvalidBits;       // invariant: S(lo) >= T > S(hi)
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      uint64_t s = 0;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) s += (bits[e] >= mid) ? w[e] : 0;
+      s = warp_sum_u64(s);
+      if (s >= T) lo = mid;
+      else hi = mid;
+    }
+    tb = lo;
+    uint64_t above = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) above += (bits[e] > tb) ? w[e] : 0;
+    above = warp_sum_u64(above);
+    const uint64_t ww = fixed_weight(tb);     // > 0 because S(tb) > S(tb + 1)
+    const uint64_t rest = T - above;
+    need = static_cast<uint32_t>((rest + ww - 1) / ww);
+  }
+  // emit in ascending index order
+  int base = 0;
+  uint32_t ties_before = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int idx = e * 32 + lane;
+    const bool present = idx < nB;
+    const bool tie = present && bits[e] == tb;
+    const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+    const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+    const bool keep = present && (bits[e] > tb || (tie && rank < need));
+    const uint32_t kmask = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[base + __popc(kmask & lt_mask)] = idx;
+    base += __popc(kmask);
+    ties_before += __popc(tmask);
+  }
+  if (lane == 0) counts[row] = base;
+}
+
+// ---------------------------------------------------------------- head scope
+// Weighted MSD radix select over 30 significant bits in three 10-bit digits.
+struct HeadState {
+  unsigned long long W, T, above;
+  unsigned int prefix;      // resolved high digits so far
+  unsigned int maxbits;
+  int bad;
+  int resolved;             // 1: tb/need final (T == 0 case)
+  int keep_all;
+  unsigned int tb;
+  unsigned int need;
+  int pad;
+};
+
+constexpr int kDigitBits = 10;
+constexpr int kBins = 1 << kDigitBits;
+
+// pass 0..2: histogram of weights by digit among elements whose higher digits
+// match the resolved prefix.  grid (chunks, G), 256 threads.
+__global__ void head_hist_kernel(const float* __restrict__ scores, long long seg_len, int pass,
+                                 unsigned long long* __restrict__ hist, HeadState* __restrict__ st) {
+  __shared__ unsigned long long sh[kBins];
+  __shared__ unsigned int smax;
+  __shared__ int sbad;
+  const int g = blockIdx.y;
+  HeadState* s = st + g;
+  if (pass > 0 && (s->resolved || s->keep_all)) return;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) sh[i] = 0;
+  if (threadIdx.x == 0) {
+    smax = 0;
+    sbad = 0;
+  }
+  __syncthreads();
+  const int shift = 20 - kDigitBits * pass;
+  const unsigned int prefix = (pass > 0) ? s->prefix : 0u;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + static_cast<long long>(g) * seg_len;
+  unsigned int lmax = 0;
+  int lbad = 0;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < seg_len;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint32_t b = __ldg(x + i);
+    if (b >= kInvalidBits) {
+      lbad = 1;
+      continue;
+    }
+    if (pass == 0) lmax = max(lmax, b);
+    if (pass > 0 && (b >> (shift + kDigitBits)) != prefix) continue;
+    const uint64_t w = fixed_weight(b);
+    if (w) atomicAdd(&sh[(b >> shift) & (kBins - 1)], static_cast<unsigned long long>(w));
+  }
+  if (pass == 0) {
+    atomicMax(&smax, lmax);
+    if (lbad) sbad = 1;
+  }
+  __syncthreads();
+  unsigned long long* gh = hist + static_cast<long long>(g) * kBins;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
+    if (sh[i]) atomicAdd(gh + i, sh[i]);
+  if (threadIdx.x == 0 && pass == 0) {
+    atomicMax(&s->maxbits, smax);
+    if (sbad) atomicExch(&s->bad, 1);
+  }
+}
+
+// After pass k: pick the digit where the weight at or above crosses T.
+// grid G, kBins threads.  Clears the histogram for the next pass.
+__global__ void head_find_kernel(int pass, uint32_t Pfix, int keep_all, unsigned long long* __restrict__ hist,
+                                 HeadState* __restrict__ st, int32_t* __restrict__ status) {
+  __shared__ unsigned long long suf[kBins];
+  const int g = blockIdx.x;
+  const int t = threadIdx.x;
+  HeadState* s = st + g;
+  if (pass > 0 && (s->resolved || s->keep_all)) return;
+  unsigned long long* gh = hist + static_cast<long long>(g) * kBins;
+  const unsigned long long v = gh[t];
+  gh[t] = 0;
+  // inclusive suffix sum: suf[t] = sum_{u >= t} v[u]
+  suf[t] = v;
+  __syncthreads();
+  for (int o = 1; o < kBins; o <<= 1) {
+    const unsigned long long add = (t + o < kBins) ? suf[t + o] : 0ull;
+    __syncthreads();
+    suf[t] += add;
+    __syncthreads();
+  }
+  __shared__ int done;
+  if (t == 0) {
+    done = 0;
+    if (pass == 0) {
+      s->W = suf[0];
+      if (s->bad) {
+        raise_status(status, LBSA_ERR_INVALID_SCORES);
+        s->keep_all = 1;
+        done = 1;
+      } else if (keep_all) {
+        s->keep_all = 1;
+        done = 1;
+      } else {
+        const unsigned __int128 num = static_cast<unsigned __int128>(suf[0]) * Pfix + ((1u << 24) - 1);
+        s->T = static_cast<unsigned long long>(num >> 24);
+        s->above = 0;
+        s->prefix = 0;
+        if (s->T == 0) {
+          s->resolved = 1;
+          s->tb = s->maxbits;
+          s->need = 1;
+          done = 1;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (done) return;
+  const unsigned long long T = s->T;
+  const unsigned long long above = s->above;
+  // largest digit t with above + suf[t] >= T (exists: suf[0] covers everything not above)
+  const bool ok_here = above + suf[t] >= T;
+  const bool ok_next = (t + 1 < kBins) && (above + suf[t + 1] >= T);
+  __syncthreads();
+  if (ok_here && !ok_next) {
+    s->above = above + ((t + 1 < kBins) ? suf[t + 1] : 0ull);
+    s->prefix = (s->prefix << kDigitBits) | static_cast<unsigned int>(t);
+    if (pass == 2) {
+      const unsigned int tb = s->prefix;
+      s->tb = tb;
+      const unsigned long long ww = fixed_weight(tb);
+      const unsigned long long rest = T - s->above;
+      s->need = static_cast<unsigned int>((rest + ww - 1) / ww);
+      s->resolved = 1;
+    }
+  }
+}
+
+// Ties (bits == tb) per query-block row.  One warp per row.
+__global__ void head_tiecount_kernel(const float* __restrict__ scores, int G, int nB, const HeadState* __restrict__ st,
+                                     int32_t* __restrict__ tiecnt) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= static_cast<long long>(G) * nB) return;
+  const HeadState* s = st + row / nB;
+  if (s->keep_all) return;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
+  int c = 0;
+  for (int j = lane; j < nB; j += 32) c += (__ldg(x + j) == s->tb);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) tiecnt[row] = c;
+}
+
+// Exclusive scan of tie counts within each segment.  grid G, 1024 threads.
+__global__ void head_tiescan_kernel(int nB, const HeadState* __restrict__ st, int32_t* __restrict__ tiecnt) {
+  __shared__ int buf[1024];
+  __shared__ int carry;
+  const int g = blockIdx.x;
+  if (st[g].keep_all) return;
+  int32_t* c = tiecnt + static_cast<long long>(g) * nB;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < nB; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int v = (i < nB) ? c[i] : 0;
+    buf[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int add = (threadIdx.x >= o) ? buf[threadIdx.x - o] : 0;
+      __syncthreads();
+      buf[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (i < nB) c[i] = carry + buf[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += buf[1023];
+    __syncthreads();
+  }
+}
+
+// Emit kept pairs per query-block row (ascending key block).  One warp per row.
+__global__ void head_emit_kernel(const float* __restrict__ scores, int G, int nB, const HeadState* __restrict__ st,
+                                 const int32_t* __restrict__ tiebase, int32_t* __restrict__ counts,
+                                 int32_t* __restrict__ cols) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= static_cast<long long>(G) * nB) return;
+  const HeadState* s = st + row / nB;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
+  int32_t* out = cols + row * nB;
+  if (s->keep_all) {
+    for (int j = lane; j < nB; j += 32) out[j] = j;
+    if (lane == 0) counts[row] = nB;
+    return;
+  }
+  const uint32_t tb = s->tb, need = s->need;
+  uint32_t ties_before = static_cast<uint32_t>(tiebase[row]);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int base = 0;
+  for (int j0 = 0; j0 < nB; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t b = (j < nB) ? __ldg(x + j) : 0u;
+    const bool tie = (j < nB) && b == tb;
+    const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+    const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+    const bool keep = (j < nB) && (b > tb || (tie && rank < need));
+    const uint32_t kmask = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[base + __popc(kmask & lt_mask)] = j;
+    base += __popc(kmask);
+    ties_before += __popc(tmask);
+  }
+  if (lane == 0) counts[row] = base;
+}
+
+// ---------------------------------------------------------------- CSR export / import
+__global__ void export_scan_kernel(const int32_t* __restrict__ counts, long long R, int32_t* __restrict__ row_ptr,
+                                   int32_t* __restrict__ nnz) {
+  __shared__ int buf[1024];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (long long base = 0; base < R; base += 1024) {
+    const long long i = base + threadIdx.x;
+    const int v = (i < R) ? counts[i] : 0;
+    buf[threadIdx.x] = v;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int add = (threadIdx.x >= o) ? buf[threadIdx.x - o] : 0;
+      __syncthreads();
+      buf[threadIdx.x] += add;
+      __syncthreads();
+    }
+    if (i < R) row_ptr[i] = carry + buf[threadIdx.x] - v;
+    __syncthreads();
+    if (threadIdx.x == 1023) carry += buf[1023];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    row_ptr[R] = carry;
+    *nnz = carry;
+  }
+}
+
+__global__ void export_copy_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ cols, long long R,
+                                   int nB, const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;
+  const int n = counts[row];
+  const int32_t* src = cols + row * nB;
+  int32_t* dst = col + row_ptr[row];
+  for (int t = lane; t < n; t += 32) dst[t] = src[t];
+}
+
+__global__ void from_csr_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col, long long R,
+                                int nB, int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+                                int32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;
+  const int a = row_ptr[row], n = row_ptr[row + 1] - a;
+  if (n < 0 || n > nB) {
+    if (lane == 0) {
+      raise_status(status, LBSA_ERR_BAD_INDEX);
+      counts[row] = 0;
+    }
+    return;
+  }
+  bool bad = false;
+  for (int t = lane; t < n; t += 32) {
+    const int c = col[a + t];
+    bad |= (c < 0 || c >= nB);
+    cols[row * nB + t] = c;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(status, LBSA_ERR_BAD_INDEX);
+  if (lane == 0) counts[row] = n;
+}
+
+inline uint32_t fixed_p(double p) {
+  return static_cast<uint32_t>(std::nearbyint(p * 16777216.0));   // ties to even in the default mode
+}
+
+}  // namespace
+
+cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s) {
+  const uint32_t P = fixed_p(p);
+  const int keep_all = p >= 1.0 ? 1 : 0;
+  const int threads = 256;
+  const long long blocks = (static_cast<long long>(R) * 32 + threads - 1) / threads;
+  dim3 grid(static_cast<unsigned>(blocks));
+#define LBSA_SEL(EPL)                                                                                       \
+  select_row_kernel<EPL><<<grid, threads, 0, s>>>(scores, R, nB, P, keep_all, bs->counts, bs->cols, bs->status)
+  if (nB <= 32) LBSA_SEL(1);
+  else if (nB <= 64) LBSA_SEL(2);
+  else if (nB <= 128) LBSA_SEL(4);
+  else if (nB <= 256) LBSA_SEL(8);
+  else if (nB <= 512) LBSA_SEL(16);
+  else if (nB <= 1024) LBSA_SEL(32);
+  else return cudaErrorInvalidValue;
+#undef LBSA_SEL
+  return cudaGetLastError();
+}
+
+size_t select_head_workspace_bytes(int B, int H, int nB) {
+  const size_t G = static_cast<size_t>(B) * H;
+  return G * kBins * sizeof(unsigned long long) + G * sizeof(HeadState) + G * nB * sizeof(int32_t) + 256;
+}
+
+cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs, void* ws,
+                               cudaStream_t s) {
+  const int G = B * H;
+  const long long seg = static_cast<long long>(nB) * nB;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(ws);
+  HeadState* st = reinterpret_cast<HeadState*>(hist + static_cast<size_t>(G) * kBins);
+  int32_t* tie = reinterpret_cast<int32_t*>(st + G);
+  cudaError_t e = cudaMemsetAsync(ws, 0, static_cast<size_t>(G) * kBins * sizeof(unsigned long long) +
+                                             static_cast<size_t>(G) * sizeof(HeadState), s);
+  if (e != cudaSuccess) return e;
+  const uint32_t P = fixed_p(p);
+  const int keep_all = p >= 1.0 ? 1 : 0;
+  const int chunks = static_cast<int>(std::min<long long>(64, (seg + 4095) / 4096));
+  for (int pass = 0; pass < 3; ++pass) {
+    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
+    head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, bs->status);
+  }
+  const long long rows = static_cast<long long>(G) * nB;
+  const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie);
+  head_tiescan_kernel<<<G, 1024, 0, s>>>(nB, st, tie);
+  head_emit_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie, bs->counts, bs->cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col, int32_t* nnz_dev,
+                              cudaStream_t s) {
+  const long long R = static_cast<long long>(bs->B) * bs->H * bs->nB;
+  export_scan_kernel<<<1, 1024, 0, s>>>(bs->counts, R, row_ptr, nnz_dev);
+  export_copy_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, s>>>(bs->counts, bs->cols, R, bs->nB,
+                                                                               row_ptr, col);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blockset* bs, cudaStream_t s) {
+  const long long R = static_cast<long long>(bs->B) * bs->H * bs->nB;
+  from_csr_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, s>>>(row_ptr, col, R, bs->nB, bs->counts,
+                                                                             bs->cols, bs->status);
+  return cudaGetLastError();
+}
+
+}  // namespace lbsa

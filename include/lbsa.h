@@ -1,0 +1,213 @@
+/*
+ * lbsa.h -- C ABI of liblbsa, block-sparse self-attention over 3D video token
+ * grids on NVIDIA B200 (sm_100a).
+ *
+ * The path has three stages, each one call below:
+ *   1. lbsa_score  -- per (head, query block) block scores: the exact block
+ *      attention mass of one dense softmax pass (LoSA abstract, scholarbro.com
+ *      author page of C. Sun) or the block-mean proxy (VMoBA review on
+ *      pith.science, arXiv 2506.23858, "What carries the argument").
+ *   2. lbsa_select -- mass-threshold selection: sort the scores, accumulate,
+ *      keep the smallest key-block set whose retained mass reaches p (LoSA
+ *      abstract; VMoBA review, circularity check: smallest k' whose cumulative
+ *      normalized similarity reaches tau), per query-block row (LoSA) or over
+ *      all block pairs of a head (VMoBA global selection).  The result is a
+ *      blockset that can be frozen and reused by later calls (LoSA abstract:
+ *      the frozen block indices are reused for all remaining steps).
+ *   3. lbsa_attend -- block-sparse flash attention that visits only the kept
+ *      key blocks (VMoBA review: only the selected blocks contribute their
+ *      actual key-value pairs).
+ * plus lbsa_permute / lbsa_partition_perm for the 1D / 2D / 3D block
+ * partitions of the token grid (VMoBA review: layer-wise cyclic 1D-2D-3D
+ * partition).
+ *
+ * Conventions shared by every call
+ *   - Pointers named q, k, v, out, scores, lse, perm, x, y are DEVICE pointers
+ *     owned by the caller; the library never frees them.  All work is
+ *     enqueued on the caller's CUDA stream (`stream`, a cudaStream_t; NULL is
+ *     the legacy default stream) and returns without synchronising unless a
+ *     function says otherwise.
+ *   - A return value is an lbsa_status.  Host-side validation failures return
+ *     LBSA_ERR_INVALID_ARG / LBSA_ERR_UNSUPPORTED before anything is launched;
+ *     lbsa_last_error() then holds a one-line reason (thread-local).
+ *   - Errors found on the device (an out-of-range block index, invalid scores,
+ *     a wait that ran out) are recorded in the blockset's device status word
+ *     (lbsa_get_status) or in the library's per-device status word
+ *     (lbsa_device_status); kernels never trap.
+ *   - Tensors are [B, H, rows, d] with d contiguous (stride 1) and element
+ *     strides stride_b, stride_h, stride_n given in lbsa_qkv_desc; rows
+ *     0..N_valid-1 are tokens in block order (block i = rows i*block ..
+ *     i*block+block-1).  A partial last block is allowed: rows >= N_valid are
+ *     never read and never written.  Base pointers and the byte sizes of
+ *     stride_b, stride_h, stride_n must be multiples of 16.
+ */
+#ifndef LBSA_H
+#define LBSA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LBSA_OK = 0,
+  LBSA_ERR_INVALID_ARG = 1,     /* bad pointer, shape, stride or parameter        */
+  LBSA_ERR_UNSUPPORTED = 2,     /* valid but not built (e.g. d not in {64,128})   */
+  LBSA_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed               */
+  LBSA_ERR_OOM = 4,             /* device allocation failed                        */
+  LBSA_ERR_BAD_INDEX = 5,       /* device: a block index outside [0, nB)           */
+  LBSA_ERR_INVALID_SCORES = 6,  /* device: a score NaN, negative or >= 2           */
+  LBSA_ERR_TIMEOUT = 7          /* device: a bounded wait ran out                  */
+} lbsa_status;
+
+typedef enum { LBSA_BF16 = 0, LBSA_F32 = 1 } lbsa_dtype;
+typedef enum { LBSA_SCORE_EXACT_MASS = 0, LBSA_SCORE_MEANPOOL = 1 } lbsa_score_mode;
+typedef enum { LBSA_SCOPE_ROW = 0, LBSA_SCOPE_HEAD = 1 } lbsa_scope;
+typedef enum {
+  LBSA_PART_RASTER = 0,         /* identity                                        */
+  LBSA_PART_1D = 1,             /* temporal rows: t fastest                        */
+  LBSA_PART_2D = 2,             /* per-frame th x tw spatial tiles                 */
+  LBSA_PART_3D = 3              /* tt x th x tw spatio-temporal tiles              */
+} lbsa_partition;
+
+typedef struct {
+  int32_t B, H;                 /* batch, heads                                    */
+  int32_t N_valid;              /* tokens per (batch, head); rows >= N_valid are padding */
+  int32_t d;                    /* head dim: 64 or 128                             */
+  int32_t dtype;                /* lbsa_dtype of q, k, v and out                   */
+  int32_t reserved;
+  int64_t stride_b, stride_h, stride_n;   /* element strides; the d stride is 1   */
+} lbsa_qkv_desc;
+
+/* Opaque, library-owned selection result: per query-block row r =
+ * (b*H + h)*nB + i the ascending list of kept key-block ids, plus a device
+ * status word.  Read-only once built; safe to reuse across any number of
+ * lbsa_attend calls (the frozen indices of LoSA). */
+typedef struct lbsa_blockset lbsa_blockset;
+
+/* Stage 1: block scores.
+ * LoSA abstract (exact mass) / VMoBA review "What carries the argument"
+ * (block-mean proxy).
+ *   q, k    [B, H, N_valid, d] per desc (bf16 or fp32)
+ *   block   tokens per block, 64 or 128 (same for queries and keys)
+ *   mode    LBSA_SCORE_EXACT_MASS: scores[b,h,i,j] = mean over the valid
+ *           query rows r of block i of sum over valid keys c of block j of
+ *           softmax_c(q_r . k_c / sqrt(d)); every row of a head sums to 1.
+ *           LBSA_SCORE_MEANPOOL: qbar_i, kbar_j = means of the valid tokens of
+ *           the blocks (fp32), s_ij = qbar_i . kbar_j / sqrt(d),
+ *           scores[b,h,:,:] = softmax over all nB*nB pairs of the head.
+ *   scores  out: fp32 [B, H, nB, nB] contiguous, nB = ceil(N_valid / block)
+ *   lse     optional out (exact mode only; NULL to skip): fp32 [B, H, N_valid]
+ *           contiguous, natural-log log-sum-exp of each query row of the dense
+ *           pass.
+ * The exact mode is a two-sweep dense pass (tensor cores for bf16). */
+int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t block,
+               int32_t mode, float* scores, float* lse, void* stream);
+
+/* Stage 2: mass-threshold selection into a new blockset.
+ * LoSA abstract (per head and query block, smallest set meeting the
+ * threshold); VMoBA review (global selection over a head; threshold tau;
+ * rows may come out empty).
+ *   scores  fp32 [B, H, nB, nB] contiguous device array, 0 <= x < 2
+ *   block   tokens per block the scores were computed with (64 or 128)
+ *   p       threshold in (0, 1]; p = 1 keeps every block (dense)
+ *   scope   LBSA_SCOPE_ROW: one decision per (b, h, query block), at least
+ *           one block kept per row.  LBSA_SCOPE_HEAD: one decision over the
+ *           nB*nB pairs of each (b, h), at least one pair per head; rows may
+ *           be empty.
+ *   out     receives a new blockset (free with lbsa_free).
+ * Rule, exact and order-independent: w = floor(x * 2^32), W = sum w,
+ * P = round_half_even(p * 2^24), T = ceil(P * W / 2^24); order by score
+ * descending, then flat index ascending; keep the shortest prefix whose sum
+ * of w is >= T (at least one element).  A segment holding a NaN, negative or
+ * >= 2 score keeps all its blocks and sets LBSA_ERR_INVALID_SCORES in the
+ * blockset's status word.  The blockset's device memory is allocated
+ * stream-ordered at worst-case size (B*H*nB*(nB+1) int32); no host sync. */
+int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,
+                int32_t scope, lbsa_blockset** out, void* stream);
+
+/* Stage 3: block-sparse attention over a (frozen) blockset.
+ * VMoBA review "What carries the argument" (only selected blocks contribute
+ * their key-value pairs); LoSA abstract (frozen indices reused).
+ *   q, k, v  [B, H, N_valid, d] per desc; bf16 runs on tcgen05 tensor cores,
+ *            fp32 on CUDA cores in true fp32
+ *   bs       blockset from lbsa_select (or lbsa_blockset_from_csr) with the
+ *            same B, H and nB = ceil(N_valid / block)
+ *   out      [B, H, N_valid, d], same dtype and strides as q:
+ *            out_r = sum_{c in K_i} softmax_{c in K_i}(q_r . k_c / sqrt(d)) v_c
+ *            where K_i are the valid keys of the kept blocks of r's block.
+ *            A row whose list is empty gets 0.
+ *   lse      optional fp32 [B, H, N_valid] (natural log; -inf for empty rows).
+ * An out-of-range block id in bs is skipped and flags LBSA_ERR_BAD_INDEX in
+ * bs's status word. */
+int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc,
+                const lbsa_blockset* bs, void* out, float* lse, void* stream);
+
+/* Release a blockset (stream-ordered on the stream it was created on).  NULL is a no-op. */
+void lbsa_free(lbsa_blockset* bs);
+
+/* Describe a blockset: any output pointer may be NULL. */
+int lbsa_blockset_info(const lbsa_blockset* bs, int32_t* B, int32_t* H, int32_t* nB,
+                       int32_t* block, int32_t* scope);
+
+/* Device views of the blockset's storage (read-only; valid until lbsa_free):
+ * counts[r] = kept blocks of row r (R = B*H*nB rows); cols[r*nB + t], t <
+ * counts[r], ascending key-block ids. */
+int lbsa_blockset_views(const lbsa_blockset* bs, const int32_t** counts, const int32_t** cols);
+
+/* Compact CSR export (a helper, not on the per-call path).  row_ptr: device
+ * int32 [R + 1]; col: device int32 with room for R*nB entries; *nnz (host)
+ * receives the total.  Synchronises the stream. */
+int lbsa_blockset_export(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col, int64_t* nnz,
+                         void* stream);
+
+/* Build a blockset from a caller CSR (device int32 row_ptr [R+1], col [nnz];
+ * lists must be ascending), e.g. frozen indices saved by an earlier run.
+ * Copies the data; ids are validated on the device (status word). */
+int lbsa_blockset_from_csr(const int32_t* row_ptr, const int32_t* col, int32_t B, int32_t H,
+                           int32_t nB, int32_t block, lbsa_blockset** out, void* stream);
+
+/* Read (and with clear != 0 reset) the blockset's device status word: 0 or an
+ * lbsa_status of the first device error.  Synchronises the stream. */
+int lbsa_get_status(const lbsa_blockset* bs, int32_t* device_status, int32_t clear, void* stream);
+
+/* Per-device status word of calls that have no blockset (lbsa_score,
+ * lbsa_permute).  Synchronises the stream. */
+int lbsa_device_status(int32_t* device_status, int32_t clear, void* stream);
+
+/* Token order of a (T, Hg, Wg) grid for one block partition (VMoBA review:
+ * 1D-2D-3D partition; raster index (t*Hg + h)*Wg + w):
+ *   blocked[slot] = raster[perm[slot]], slot in [0, T*Hg*Wg).
+ * LBSA_PART_1D: t fastest.  LBSA_PART_2D: per frame, th x tw tiles in raster
+ * tile order, raster inside a tile.  LBSA_PART_3D: tt x th x tw tiles in
+ * raster tile order, raster inside a tile.  Edge tiles are truncated.
+ * on_device != 0: perm is a device pointer, filled by a kernel on stream;
+ * otherwise a host pointer, filled synchronously on the CPU. */
+int lbsa_partition_perm(int32_t T, int32_t Hg, int32_t Wg, int32_t kind, int32_t tt, int32_t th,
+                        int32_t tw, int32_t* perm, int32_t on_device, void* stream);
+
+/* Row gather / scatter of up to 3 tensors that share desc and perm:
+ *   inverse == 0:  ys[t][b,h,slot,:] = xs[t][b,h,perm[slot],:]
+ *   inverse != 0:  ys[t][b,h,perm[slot],:] = xs[t][b,h,slot,:]
+ * for slot < desc->N_valid; perm (device int32 [N_valid]) must be a
+ * permutation of [0, N_valid).  x and y may not alias. */
+int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const int32_t* perm,
+                 const lbsa_qkv_desc* desc, int32_t inverse, void* stream);
+
+/* Self-test of the bounded-wait machinery: one kernel waits on an mbarrier
+ * that nothing completes, gives up after `iters` polls and writes
+ * LBSA_ERR_TIMEOUT to *device_out (device int32).  Never hangs. */
+int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream);
+
+/* Thread-local one-line reason for the last non-OK return of this thread. */
+const char* lbsa_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int lbsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LBSA_H */

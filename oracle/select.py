@@ -57,13 +57,9 @@ def _segment_keep(bits: np.ndarray, w: np.ndarray, p: float) -> np.ndarray:
     idx = np.arange(n)
     # order: bits descending, then index ascending (lexsort's last key is primary)
     order = np.lexsort((idx, -bits.astype(np.int64)))
-    csum = 0
-    k = n
-    for pos in range(n):
-        csum += int(w[order[pos]])
-        if csum >= T:
-            k = pos + 1
-            break
+    csum = np.cumsum(w[order])              # int64, exact: n * 2^33 < 2^63
+    hit = np.nonzero(csum >= T)[0]
+    k = int(hit[0]) + 1 if len(hit) else n
     k = max(k, 1)
     return np.sort(order[:k])
 

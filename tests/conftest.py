@@ -4,8 +4,17 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+TESTS = os.path.dirname(os.path.abspath(__file__))
+if TESTS not in sys.path:
+    sys.path.insert(0, TESTS)
 
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    config.addinivalue_line("markers", "slow: larger CPU cases")
+
+
+def pytest_sessionstart(session):
+    # liblbsa.so is built in-tree (nvcc cross-compiles without a GPU); this is
+    # a no-op when the library is current.
+    from block_sparse_attention_16_b200.build import build
+    build()

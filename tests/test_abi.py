@@ -1,0 +1,120 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared
+symbol, rejects bad arguments before launching anything, and its host-side
+partition order matches the oracle bit for bit."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import block_sparse_attention_16_b200 as lbsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lbsa.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lbsa_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = lbsa.load_library()
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lbsa.lbsa_version() == 100
+
+
+def _desc(**kw):
+    d = dict(B=1, H=2, N_valid=256, d=64, dtype=1, reserved=0, stride_b=2 * 256 * 64, stride_h=256 * 64, stride_n=64)
+    d.update(kw)
+    return lbsa._Desc(**d)
+
+
+FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), lbsa.LBSA_ERR_UNSUPPORTED),
+    (dict(N_valid=0), lbsa.LBSA_ERR_INVALID_ARG),
+    (dict(dtype=7), lbsa.LBSA_ERR_INVALID_ARG),
+    (dict(stride_n=60), lbsa.LBSA_ERR_INVALID_ARG),
+    (dict(stride_n=65), lbsa.LBSA_ERR_INVALID_ARG),
+])
+def test_score_rejects_bad_desc(kw, code):
+    lib = lbsa.load_library()
+    d = _desc(**kw)
+    rc = lib.lbsa_score(FAKE, FAKE, ctypes.byref(d), 64, 0, FAKE, None, None)
+    assert rc == code
+    assert lbsa.lbsa_last_error()
+
+
+def test_score_rejects_bad_block_mode_and_pointers():
+    lib = lbsa.load_library()
+    d = _desc()
+    assert lib.lbsa_score(FAKE, FAKE, ctypes.byref(d), 96, 0, FAKE, None, None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_score(FAKE, FAKE, ctypes.byref(d), 64, 9, FAKE, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_score(None, FAKE, ctypes.byref(d), 64, 0, FAKE, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_score(ctypes.c_void_p(0x10004), FAKE, ctypes.byref(d), 64, 0, FAKE, None, None) == \
+        lbsa.LBSA_ERR_INVALID_ARG
+    # lse is only defined for the exact mode
+    assert lib.lbsa_score(FAKE, FAKE, ctypes.byref(d), 64, 1, FAKE, FAKE, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("p", [0.0, -0.5, 1.5, float("nan")])
+def test_select_rejects_bad_p(p):
+    lib = lbsa.load_library()
+    h = ctypes.c_void_p()
+    assert lib.lbsa_select(FAKE, 1, 1, 4, 64, p, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert not h.value
+
+
+def test_select_rejects_bad_scope_block_and_size():
+    lib = lbsa.load_library()
+    h = ctypes.c_void_p()
+    assert lib.lbsa_select(FAKE, 1, 1, 4, 64, 0.9, 5, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select(FAKE, 1, 1, 4, 32, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select(FAKE, 1, 1, 2000, 64, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select(FAKE, 1, 1, 0, 64, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select(FAKE, 1, 1, 4, 64, 0.9, 0, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+def test_attend_rejects_null_blockset_and_permute_aliasing():
+    lib = lbsa.load_library()
+    d = _desc()
+    assert lib.lbsa_attend(FAKE, FAKE, FAKE, ctypes.byref(d), None, FAKE, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+    xs = (ctypes.c_void_p * 1)(0x10000)
+    assert lib.lbsa_permute(xs, xs, 1, FAKE, ctypes.byref(d), 0, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_permute(xs, xs, 4, FAKE, ctypes.byref(d), 0, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+def test_free_null_is_noop_and_info_rejects_null():
+    lib = lbsa.load_library()
+    lib.lbsa_free(None)
+    assert lib.lbsa_blockset_info(None, None, None, None, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (21, 30, 52), (5, 7, 9), (33, 45, 80)])
+def test_host_partition_perm_matches_oracle(grid):
+    T, H, W = grid
+    assert np.array_equal(lbsa.lbsa_partition_perm(T, H, W, "raster").numpy(), oracle.perm_raster(T, H, W))
+    assert np.array_equal(lbsa.lbsa_partition_perm(T, H, W, "1d").numpy(), oracle.perm_1d_temporal(T, H, W))
+    assert np.array_equal(lbsa.lbsa_partition_perm(T, H, W, "2d", frame_tile=(8, 8)).numpy(),
+                          oracle.perm_2d_frame_tiles(T, H, W, 8, 8))
+    assert np.array_equal(lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4)).numpy(),
+                          oracle.perm_3d_tiles(T, H, W, 4, 4, 4))
+    assert np.array_equal(lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(3, 5, 2)).numpy(),
+                          oracle.perm_3d_tiles(T, H, W, 3, 5, 2))
+
+
+def test_partition_perm_rejects_bad_args():
+    lib = lbsa.load_library()
+    buf = (ctypes.c_int32 * 8)()
+    assert lib.lbsa_partition_perm(0, 2, 2, 0, 1, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_partition_perm(2, 2, 2, 9, 1, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_partition_perm(2, 2, 2, 3, 0, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG

@@ -1,0 +1,255 @@
+"""GPU parity on small shapes: every path of the C ABI against the fp64 oracle.
+
+Shapes span several 128-row tiles, ragged last blocks, both block sizes, both
+head dims, batch > 1, empty rows, p = 1 (dense) and the status-word paths.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import block_sparse_attention_16_b200 as lbsa
+from block_sparse_attention_16_b200.workload import get_workload, make_qkv, small_workload
+from parity import assert_csr_equal, assert_out_close, assert_scores_close, gpu_csr, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.set_device(0)
+    lbsa.lbsa_device_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def _pipeline(wl, p, scope="row", mode="exact"):
+    q, k, v = (x.cuda() for x in make_qkv(wl))
+    scores, lse_d = (lbsa.lbsa_score(q, k, wl.block, mode=mode, want_lse=True) if mode == "exact"
+                     else (lbsa.lbsa_score(q, k, wl.block, mode=mode), None))
+    bs = lbsa.lbsa_select(scores, wl.block, p, scope)
+    out, lse = lbsa.lbsa_attend(q, k, v, bs, want_lse=True)
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_device_status() == 0
+    assert lbsa.lbsa_get_status(bs) == 0
+    return q, k, v, scores, lse_d, bs, out, lse
+
+
+# ------------------------------------------------------------------ plumbing
+def test_bounded_wait_reports_timeout():
+    assert lbsa.lbsa_selftest_wait(2000) == lbsa.LBSA_ERR_TIMEOUT
+
+
+@pytest.mark.parametrize("grid", [(4, 8, 8), (21, 30, 52), (5, 7, 9)])
+def test_device_partition_perm_matches_oracle(grid):
+    T, H, W = grid
+    for kind, ref in (("1d", oracle.perm_1d_temporal(T, H, W)), ("2d", oracle.perm_2d_frame_tiles(T, H, W)),
+                      ("3d", oracle.perm_3d_tiles(T, H, W)), ("raster", oracle.perm_raster(T, H, W))):
+        got = lbsa.lbsa_partition_perm(T, H, W, kind, device="cuda").cpu().numpy()
+        assert np.array_equal(got, ref), kind
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_permute_gather_scatter(dtype, d):
+    T, H, W = 5, 7, 9
+    n = T * H * W
+    g = torch.Generator(device="cuda").manual_seed(3)
+    xs = [torch.randn(2, 3, n, d, generator=g, device="cuda").to(dtype) for _ in range(3)]
+    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", device="cuda")
+    ys = lbsa.lbsa_permute(xs, perm)
+    pl = perm.long()
+    for x, y in zip(xs, ys):
+        assert torch.equal(y, x[:, :, pl])
+    back = lbsa.lbsa_permute(ys, perm, inverse=True)
+    for x, b in zip(xs, back):
+        assert torch.equal(b, x)
+
+
+# ------------------------------------------------------------------ fp32 path (true fp32)
+@pytest.mark.parametrize("p", [0.5, 0.9, 0.99, 1.0])
+def test_tiny_fp32_pipeline(p):
+    wl = get_workload("tiny")
+    q, k, v, scores, lse_d, bs, out, lse = _pipeline(wl, p)
+    qh, kh, vh = host(q), host(k), host(v)
+    assert_scores_close(host(scores), oracle.block_mass(qh, kh, wl.n_valid, wl.block))
+    _, ref_lse = oracle.dense_attention(qh, kh, vh, wl.n_valid)
+    assert np.max(np.abs(host(lse_d) - ref_lse)) <= 1e-5
+    csr = gpu_csr(bs)
+    assert_csr_equal(csr, oracle.select_contract(host(scores), p, "row"))
+    ref_o, ref_l = oracle.sparse_attention(qh, kh, vh, wl.n_valid, wl.block, *csr)
+    assert_out_close(host(out), ref_o[:, :, :wl.n_valid], torch.float32)
+    assert np.max(np.abs(host(lse) - ref_l[:, :, :wl.n_valid])) <= 1e-5
+
+
+def test_fp32_ragged_multi_batch():
+    wl = small_workload("f32r", 2, 2, 128, (3, 5, 9), 64, dtype="f32", wid=101)   # 135 tokens, last block 7
+    q, k, v, scores, _, bs, out, lse = _pipeline(wl, 0.95)
+    qh, kh, vh = host(q), host(k), host(v)
+    assert_scores_close(host(scores), oracle.block_mass(qh, kh, wl.n_valid, wl.block))
+    csr = gpu_csr(bs)
+    assert_csr_equal(csr, oracle.select_contract(host(scores), 0.95, "row"))
+    ref_o, _ = oracle.sparse_attention(qh, kh, vh, wl.n_valid, wl.block, *csr)
+    assert_out_close(host(out), ref_o[:, :, :wl.n_valid], torch.float32)
+
+
+# ------------------------------------------------------------------ bf16 tensor-core path
+BF16_CASES = [
+    # name, B, H, d, grid, block
+    ("b64_d128_ragged", 2, 2, 128, (3, 8, 12), 64),       # 288 tokens: 5 blocks, last 32 valid, 3 tiles
+    ("b128_d128_ragged", 1, 3, 128, (4, 9, 10), 128),     # 360 tokens: 3 blocks, last 104 valid
+    ("b64_d64_ragged", 1, 2, 64, (5, 6, 7), 64),          # 210 tokens: 4 blocks, last 18 valid
+    ("b64_d128_16blk", 1, 2, 128, (4, 16, 16), 64),       # 1024 tokens: 16 blocks, 8 tiles
+    ("b128_d64_odd", 2, 1, 64, (3, 7, 31), 128),          # 651 tokens: 6 blocks, last 11 valid
+]
+
+
+@pytest.mark.parametrize("case", BF16_CASES, ids=lambda c: c[0])
+@pytest.mark.parametrize("p", [0.9, 0.99])
+def test_bf16_pipeline(case, p):
+    name, B, H, d, grid, block = case
+    wl = small_workload(name, B, H, d, grid, block, dtype="bf16", wid=110 + BF16_CASES.index(case))
+    q, k, v, scores, lse_d, bs, out, lse = _pipeline(wl, p)
+    qh, kh, vh = host(q), host(k), host(v)
+    assert_scores_close(host(scores), oracle.block_mass(qh, kh, wl.n_valid, wl.block))
+    _, ref_dl = oracle.dense_attention(qh, kh, vh, wl.n_valid)
+    assert np.max(np.abs(host(lse_d) - ref_dl)) <= 1e-3
+    csr = gpu_csr(bs)
+    assert_csr_equal(csr, oracle.select_contract(host(scores), p, "row"))
+    ref_o, ref_l = oracle.sparse_attention(qh, kh, vh, wl.n_valid, wl.block, *csr)
+    assert_out_close(host(out), ref_o[:, :, :wl.n_valid], torch.bfloat16)
+    assert np.max(np.abs(host(lse) - ref_l[:, :, :wl.n_valid])) <= 1e-2
+
+
+@pytest.mark.parametrize("case", BF16_CASES[:3], ids=lambda c: c[0])
+def test_bf16_dense_p1_equals_dense_attention(case):
+    name, B, H, d, grid, block = case
+    wl = small_workload(name, B, H, d, grid, block, dtype="bf16", wid=120)
+    q, k, v, scores, _, bs, out, lse = _pipeline(wl, 1.0)
+    rp, col = gpu_csr(bs)
+    assert np.all(np.diff(rp) == wl.n_blocks)
+    ref_o, ref_l = oracle.dense_attention(host(q), host(k), host(v), wl.n_valid)
+    assert_out_close(host(out), ref_o, torch.bfloat16)
+    assert np.max(np.abs(host(lse) - ref_l)) <= 1e-2
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("block", [64, 128])
+def test_hand_built_lists_with_empty_rows(dtype, block):
+    wl = small_workload("csr", 1, 2, 128, (4, 10, 16), block, dtype=dtype, wid=130)    # 640 tokens
+    q, k, v = (x.cuda() for x in make_qkv(wl))
+    nB = wl.n_blocks
+    rng = np.random.default_rng(block)
+    rows = []
+    for h in range(wl.H):
+        for i in range(nB):
+            r = rng.random()
+            if r < 0.25:
+                rows.append(np.zeros(0, dtype=np.int64))                      # empty row
+            elif r < 0.5:
+                rows.append(np.array([int(rng.integers(nB))]))                 # single block
+            else:
+                rows.append(np.sort(rng.choice(nB, size=int(rng.integers(1, nB + 1)), replace=False)))
+    rp, col = oracle.csr_from_rows(rows)
+    bs = lbsa.lbsa_blockset_from_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(),
+                                     wl.B, wl.H, nB, block)
+    out, lse = lbsa.lbsa_attend(q, k, v, bs, want_lse=True)
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs) == 0
+    assert_csr_equal(gpu_csr(bs), (rp, col))
+    ref_o, ref_l = oracle.sparse_attention(host(q), host(k), host(v), wl.n_valid, block, rp, col)
+    assert_out_close(host(out), ref_o[:, :, :wl.n_valid], q.dtype)
+    gl = host(lse)
+    rl = ref_l[:, :, :wl.n_valid]
+    assert np.array_equal(np.isneginf(gl), np.isneginf(rl))
+    fin = np.isfinite(rl)
+    assert np.max(np.abs(gl[fin] - rl[fin])) <= 1e-2
+    empty = np.isneginf(rl)
+    assert np.all(host(out)[empty] == 0)
+
+
+def test_bad_block_index_is_flagged_and_skipped():
+    wl = small_workload("bad", 1, 1, 128, (2, 8, 16), 64, dtype="bf16", wid=131)   # 256 tokens, 4 blocks
+    q, k, v = (x.cuda() for x in make_qkv(wl))
+    rows = [np.array([0, 1]), np.array([1, 7]), np.array([2]), np.array([0, 3])]   # 7 is out of range
+    rp, col = oracle.csr_from_rows(rows)
+    bs = lbsa.lbsa_blockset_from_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(), 1, 1, 4, 64)
+    out = lbsa.lbsa_attend(q, k, v, bs)
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs, clear=True) == lbsa.LBSA_ERR_BAD_INDEX
+    assert lbsa.lbsa_get_status(bs) == 0
+    clean = [np.array([0, 1]), np.array([1]), np.array([2]), np.array([0, 3])]
+    crp, ccol = oracle.csr_from_rows(clean)
+    ref_o, _ = oracle.sparse_attention(host(q), host(k), host(v), wl.n_valid, 64, crp, ccol)
+    assert_out_close(host(out), ref_o, torch.bfloat16)
+
+
+def test_invalid_scores_keep_all_and_flag():
+    scores = torch.full((1, 2, 8, 8), 1.0 / 8, device="cuda")
+    scores[0, 1, 3, 5] = float("nan")
+    bs = lbsa.lbsa_select(scores, 64, 0.5, "row")
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs) == lbsa.LBSA_ERR_INVALID_SCORES
+    rp, col = gpu_csr(bs)
+    counts = np.diff(rp)
+    assert counts[8 + 3] == 8                        # the poisoned row keeps everything
+    assert np.all(counts[:8] == 4)                   # 4 x 1/8 = 0.5 reaches p = 0.5
+    bs2 = lbsa.lbsa_select(scores, 64, 0.5, "head")
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs2) == lbsa.LBSA_ERR_INVALID_SCORES
+    rp2, _ = gpu_csr(bs2)
+    assert np.all(np.diff(rp2)[8:] == 8)             # the poisoned head keeps everything
+
+
+# ------------------------------------------------------------------ selection on synthetic score matrices
+@pytest.mark.parametrize("nB", [1, 4, 33, 100, 512, 929])
+@pytest.mark.parametrize("kind", ["dirichlet", "ties", "peaked"])
+def test_select_row_bit_exact(nB, kind):
+    rng = np.random.default_rng(nB)
+    H = 3
+    if kind == "dirichlet":
+        x = rng.dirichlet(np.ones(nB) * 0.3, size=(1, H, nB))
+    elif kind == "ties":
+        x = rng.choice(np.array([0.0, 1 / 64, 1 / 32, 3 / 64, 1 / 8]), size=(1, H, nB, nB))
+    else:
+        z = rng.standard_normal((1, H, nB, nB)) * 6
+        x = np.exp(z - z.max(-1, keepdims=True))
+        x /= x.sum(-1, keepdims=True)
+    x = x.astype(np.float32)
+    s = torch.from_numpy(x).cuda()
+    for p in (0.25, 0.9, 0.99, 0.999):
+        bs = lbsa.lbsa_select(s, 64, p, "row")
+        assert_csr_equal(gpu_csr(bs), oracle.select_contract(x, p, "row"))
+        assert lbsa.lbsa_get_status(bs) == 0
+
+
+@pytest.mark.parametrize("nB", [2, 16, 100, 512])
+@pytest.mark.parametrize("kind", ["softmax", "ties"])
+def test_select_head_bit_exact(nB, kind):
+    rng = np.random.default_rng(7 + nB)
+    H = 2
+    if kind == "softmax":
+        z = rng.standard_normal((1, H, nB, nB)) * 3
+        x = np.exp(z - z.max(axis=(2, 3), keepdims=True))
+        x /= x.sum(axis=(2, 3), keepdims=True)
+    else:
+        x = rng.choice(np.array([0.0, 2.0 ** -20, 2.0 ** -16, 2.0 ** -14]), size=(1, H, nB, nB))
+    x = x.astype(np.float32)
+    s = torch.from_numpy(x).cuda()
+    for p in (0.1, 0.25, 0.5, 0.9, 1.0):
+        bs = lbsa.lbsa_select(s, 64, p, "head")
+        assert_csr_equal(gpu_csr(bs), oracle.select_contract(x, p, "head"))
+        assert lbsa.lbsa_get_status(bs) == 0
+
+
+# ------------------------------------------------------------------ block-mean proxy + head scope
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_meanpool_head_scope_pipeline(dtype):
+    wl = small_workload("mp", 1, 3, 128, (4, 12, 20), 64, dtype=dtype, wid=140)   # 960 tokens: 15 blocks
+    q, k, v, scores, _, bs, out, lse = _pipeline(wl, 0.25, scope="head", mode="meanpool")
+    qh, kh, vh = host(q), host(k), host(v)
+    assert_scores_close(host(scores), oracle.meanpool_scores(qh, kh, wl.n_valid, wl.block))
+    csr = gpu_csr(bs)
+    assert_csr_equal(csr, oracle.select_contract(host(scores), 0.25, "head"))
+    ref_o, _ = oracle.sparse_attention(qh, kh, vh, wl.n_valid, wl.block, *csr)
+    assert_out_close(host(out), ref_o[:, :, :wl.n_valid], q.dtype)
