@@ -1,0 +1,391 @@
+"""Benchmark of the block-sparse video-attention hot path on B200.
+
+One step = one pass of the whole path over one Wan-like attention layer
+(B=1, H=12, d=128, 21x30x52 = 32,760 tokens, bf16, 64-token blocks):
+  3D-tile permutation of Q, K, V  ->  exact block mass (two-sweep dense pass)
+  ->  fixed-point row selection at p = 0.99  ->  block-sparse attention
+  ->  inverse permutation of O.
+Inputs are resident in HBM when timing starts (302 MB of Q/K/V per step, larger
+than the 126 MB L2, so no extra flush is needed between steps).
+
+value  = algorithmic TFLOP/s of the whole step, summed over ranks:
+         exact mass 2*N^2*d*H (one Q K^T) + attention 4*d*sum_kept(valid_q*valid_k)
+         per step, divided by the max-over-ranks device time of the K steps.
+Multi-GPU (--gpus N under torchrun): every rank runs its own layer (the path
+shards by (batch, head) with no exchange step), so scaling is weak and there is
+no data-path collective.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "block-sparse attn ms/call & achieved TFLOP/s at p=0.99, frac of B200 roofline"
+WORKLOAD = "wan"
+P = 0.99
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "source": "of measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "of fallback"}
+
+
+def attention_flops(counts, nB, block, n_valid, d):
+    """4*d*sum over kept (query block, key block) of valid_q * valid_k."""
+    valid = np.full(nB, block, dtype=np.float64)
+    valid[-1] = n_valid - (nB - 1) * block
+    c = counts.reshape(-1, nB, nB) if counts.ndim == 3 else counts
+    return 4.0 * d * float(np.einsum("gij,i,j->", c, valid, valid))
+
+
+def kept_mask(row_ptr, col, rows, nB):
+    m = np.zeros((rows, nB), dtype=np.float64)
+    r = np.repeat(np.arange(rows), np.diff(row_ptr))
+    m[r, col] = 1.0
+    return m
+
+
+class Clocks:
+    """nvidia-smi sampler for the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, path):
+        self.path = path
+        self.proc = None
+        try:
+            self.f = open(path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle (CPU) sample
+def oracle_sample(q, k, v, wl, heads_qblocks, p=P):
+    """Run the fp64 oracle on sampled (head, query block) units; returns (flops, seconds)."""
+    import oracle
+    nB, b, n, d = wl.n_blocks, wl.block, wl.n_valid, wl.d
+    flops = 0.0
+    t0 = time.perf_counter()
+    for h, qbs in heads_qblocks:
+        qh = q[:, h:h + 1].float().numpy()
+        kh = k[:, h:h + 1].float().numpy()
+        vh = v[:, h:h + 1].float().numpy()
+        mass = oracle.block_mass(qh, kh, n, b, qblocks=qbs)
+        rows = []
+        for t, i in enumerate(qbs):
+            seg = mass[:, :, t:t + 1, :].astype(np.float32)
+            rp, col = oracle.select_contract(seg, p, "row")
+            rows.append(col)
+        full = [np.zeros(0, dtype=np.int64)] * nB
+        for i, c in zip(qbs, rows):
+            full[i] = c
+        rp, col = oracle.csr_from_rows(full)
+        oracle.sparse_attention(qh, kh, vh, n, b, rp, col, qblocks=qbs)
+        for i, c in zip(qbs, rows):
+            vq = min(b, n - i * b)
+            flops += 2.0 * vq * n * d
+            vk = sum(min(b, n - j * b) for j in c)
+            flops += 4.0 * d * vq * vk
+    return flops, time.perf_counter() - t0
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv
+    wl = get_workload(WORKLOAD)
+    q, k, v = make_qkv(wl, device="cpu")
+    import oracle
+    T, H, W = wl.grid
+    perm = oracle.perm_3d_tiles(T, H, W, 4, 4, 4)
+    q, k, v = (x[:, :, torch.from_numpy(perm)] for x in (q, k, v))
+    rng = np.random.default_rng(0)
+    per_step = 4
+
+    def sample(step):
+        h = step % wl.H
+        return [(h, sorted(rng.choice(wl.n_blocks, per_step, replace=False).tolist()))]
+
+    for s in range(args.warmup):
+        oracle_sample(q, k, v, wl, sample(s))
+    tot_f, tot_t = 0.0, 0.0
+    for s in range(args.steps):
+        f, t = oracle_sample(q, k, v, wl, sample(args.warmup + s))
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    n_cores = cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": n_cores, "kind": "oracle",
+                         "sample": f"{per_step} query blocks of one head per step (exact mass row sweep, "
+                                   f"fixed-point selection, sparse attention) on the 3D-tile-ordered layer"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(wl, world):
+    T, H, W = wl.grid
+    return {"workload": f"Wan-like layer {T}x{H}x{W} ({wl.n_valid} tokens), H={wl.H}, d={wl.d}, "
+                        f"{wl.block}-token blocks, 3D 4x4x4 tiles, exact mass, p={P}",
+            "B": wl.B, "H": wl.H, "d": wl.d, "n_valid": wl.n_valid, "block": wl.block, "p": P,
+            "partition": "3d tiles 4x4x4", "l2": "inputs larger than L2 (302 MB Q/K/V per step)",
+            "parallelism": f"replicas x{world} (independent layers, no collective)"}
+
+
+# ---------------------------------------------------------------- own arm
+def run_own(args, rank, world):
+    import block_sparse_attention_16_b200 as lbsa
+    from block_sparse_attention_16_b200.build import build
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv
+
+    if rank == 0:
+        build()
+    if world > 1:
+        torch.distributed.barrier()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    lbsa.load_library()
+    wl = get_workload(WORKLOAD)
+    T, H, W = wl.grid
+    q, k, v = make_qkv(wl, device=dev)
+    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4), device=dev)
+    stream = torch.cuda.current_stream()
+    nB = wl.n_blocks
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+        if ev:
+            ev[1].record(stream)
+        scores = lbsa.lbsa_score(qp, kp, wl.block)
+        if ev:
+            ev[2].record(stream)
+        bs = lbsa.lbsa_select(scores, wl.block, P, "row")
+        if ev:
+            ev[3].record(stream)
+        op = lbsa.lbsa_attend(qp, kp, vp, bs)
+        if ev:
+            ev[4].record(stream)
+        o = lbsa.lbsa_permute([op], perm, inverse=True)[0]
+        if ev:
+            ev[5].record(stream)
+        return o, bs
+
+    for _ in range(args.warmup):
+        o, bs = step()
+    torch.cuda.synchronize()
+    rp, col = lbsa.lbsa_blockset_export(bs)
+    rp, col = rp.cpu().numpy(), col.cpu().numpy()
+    R = wl.B * wl.H * nB
+    mask = kept_mask(rp, col, R, nB).reshape(wl.B * wl.H, nB, nB)
+    att_flops = attention_flops(mask, nB, wl.block, wl.n_valid, wl.d)
+    score_flops = 2.0 * wl.n_valid ** 2 * wl.d * wl.H * wl.B
+    step_flops = att_flops + score_flops
+    density = float(mask.mean())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = Clocks(dev.index, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+                    if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/lbsa_clocks_{rank}.csv")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        o, bs = step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    stage_names = ["permute", "score", "select", "attend", "unpermute"]
+    stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(stage_names)}
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    pk = peaks()
+    att_ms = stages["attend"]
+    sc_ms = stages["score"]
+    att_tflops = att_flops / (att_ms * 1e-3) / 1e12
+    sc_tflops = score_flops / (sc_ms * 1e-3) / 1e12
+    dominant = "attend" if att_ms >= sc_ms else "score"
+    dom_flops = att_flops if dominant == "attend" else score_flops
+    dom_ms = max(att_ms, sc_ms)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    traffic = load_traffic(dominant)
+    roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": pk["bf16_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
+                "peak_source": pk["source"] + " (bf16 sustained; kernel timed inside a step)"}
+
+    # end to end through the public API: pinned host -> device, path, device -> host
+    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    qd, kd, vd = (torch.empty_like(q) for _ in range(3))
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        qp, kp, vp = lbsa.lbsa_permute([qd, kd, vd], perm)
+        scores = lbsa.lbsa_score(qp, kp, wl.block)
+        bsx = lbsa.lbsa_select(scores, wl.block, P, "row")
+        op = lbsa.lbsa_attend(qp, kp, vp, bsx)
+        ox = lbsa.lbsa_permute([op], perm, inverse=True)[0]
+        oh.copy_(ox, non_blocking=True)
+        return bsx
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    bytes_in = 3 * q.numel() * q.element_size()
+    bytes_out = q.numel() * q.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qc, kc, vc = (x[:, :, perm.long()].cpu() for x in (q, k, v))
+        rng = np.random.default_rng(1)
+        sample = [(h, sorted(rng.choice(nB, 4, replace=False).tolist())) for h in range(0, wl.H, 2)]
+        f, t = oracle_sample(qc, kc, vc, wl, sample)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
+               "sample": f"{sum(len(x[1]) for x in sample)} query blocks over {len(sample)} heads "
+                         f"(exact mass row sweep, fixed-point selection, sparse attention), {t:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
+            "stages_ms": stages, "density": density,
+            "attend": {"ms_per_call": att_ms, "tflops": att_tflops,
+                       "frac": att_tflops / pk["bf16_sustained"], "flops_per_call": att_flops},
+            "score": {"ms_per_call": sc_ms, "tflops": sc_tflops, "flops_per_call": score_flops},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * step_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": e2e_ms / args.steps,
+                    "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": bytes_out},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it covers this kernel version."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    return d.get(kernel)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        return run_own(args, rank, world)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())
