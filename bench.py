@@ -363,6 +363,37 @@ def load_traffic(kernel):
     return d.get(kernel)
 
 
+def run_profile(kernel):
+    """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
+    than L2), one warm-up pass of the path, then two launches of `kernel`."""
+    import dataclasses
+
+    import block_sparse_attention_16_b200 as lbsa
+    from block_sparse_attention_16_b200.build import build
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv
+
+    build()
+    wl = dataclasses.replace(get_workload(WORKLOAD), H=6)
+    T, H, W = wl.grid
+    q, k, v = make_qkv(wl, device="cuda")
+    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4), device="cuda")
+    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+    scores = lbsa.lbsa_score(qp, kp, wl.block)
+    bs = lbsa.lbsa_select(scores, wl.block, P, "row")
+    lbsa.lbsa_attend(qp, kp, vp, bs)
+    for _ in range(2):
+        if kernel == "attend":
+            lbsa.lbsa_attend(qp, kp, vp, bs)
+        elif kernel == "score":
+            lbsa.lbsa_score(qp, kp, wl.block, scores=scores)
+        elif kernel == "select":
+            lbsa.lbsa_select(scores, wl.block, P, "row")
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+    print(f"profile case {kernel}: ok")
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -370,7 +401,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["attend", "score", "select"],
+                    help="run the small ncu case for one kernel instead of the benchmark")
     args = ap.parse_args()
+    if args.profile:
+        return run_profile(args.profile)
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

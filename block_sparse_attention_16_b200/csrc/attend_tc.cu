@@ -14,14 +14,17 @@
 //
 // Warp roles (192 threads):
 //   warps 0-3  softmax: thread t owns tile row t = TMEM lane t.  Reads S from
-//              TMEM, keeps the running max / sum, writes P (bf16) into a
-//              128-byte-swizzled shared-memory tile, rescales O in TMEM when
-//              the running max grows by more than 2^8, and writes the output.
+//              TMEM, keeps the running max / sum, writes P (bf16, packed two
+//              per column) back over the first 32 columns of the same S
+//              buffer, rescales O in TMEM when the running max grows by more
+//              than 2^8, and writes the output.
 //   warp 4     TMA producer: Q once, then K and V 64-key tiles through a
-//              3-stage ring.
-//   warp 5     UMMA issuer: S = Q K^T (M=128, N=64, K=d) into one of two TMEM
-//              S buffers, then O += P V (M=128, N=d, K=64) into TMEM.
-// TMEM columns: [0,64) S0, [64,128) S1, [128,128+d) O.
+//              2-stage ring.
+//   warp 5     UMMA issuer: S = Q K^T (M=128, N=64, K=d, both operands in
+//              smem) into one of two TMEM S buffers, then O += P V (M=128,
+//              N=d, K=64, P read from TMEM) into TMEM.
+// TMEM columns: [0,64) S0/P0, [64,128) S1/P1, [128,128+d) O.  About 100 KB of
+// shared memory per CTA, so two CTAs (two softmax warpgroups) share an SM.
 #include "lbsa_device.cuh"
 
 namespace lbsa {
@@ -29,7 +32,7 @@ namespace {
 
 constexpr int BM = 128;           // query rows per tile
 constexpr int BK = 64;            // keys per step
-constexpr int NS = 3;             // K/V ring depth
+constexpr int NS = 2;             // K/V ring depth
 constexpr int kThreads = 192;
 constexpr int kMaxBlocks = 4096;  // nB bound (bitmap size)
 constexpr int kMaxWords = kMaxBlocks / 32;
@@ -39,12 +42,10 @@ template <int D>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BK * D * 2;
-  static constexpr int P_BYTES = BM * BK * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * KV_BYTES;
   // q_full, k_full[NS], k_empty[NS], v_full[NS], v_empty[NS], s_full[2], p_full[2], o_done[2], drain
   static constexpr int NBAR = 1 + 4 * NS + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort, n_entries, pad
@@ -81,7 +82,7 @@ __device__ __forceinline__ Bars make_bars(uint8_t* base) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const AttendArgs args, float scale_log2) {
   using L = Layout<D>;
@@ -231,7 +232,6 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK0 = smem_u32(smem + L::OFF_K);
       const uint32_t sV0 = smem_u32(smem + L::OFF_V);
-      const uint32_t sP0 = smem_u32(smem + L::OFF_P);
       bool ok = n_steps == 0 || mbar_wait(bars.q_full, 0, wl, args.status, abort_flag);
       for (int s = 0; ok && s <= n_steps; ++s) {
         if (s < n_steps) {
@@ -256,13 +256,12 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           if (!mbar_wait(bars.p_full + (j & 1), (j >> 1) & 1, wl, args.status, abort_flag)) break;
           if (!mbar_wait(bars.v_full + st, (j / NS) & 1, wl, args.status, abort_flag)) break;
           tc_fence_after();
-          const uint32_t pbase = sP0 + (j & 1) * L::P_BYTES;
+          const uint32_t pcol = tmem + (j & 1) * BK;
           const uint32_t vbase = sV0 + st * L::KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t a = smem_desc_sw128(pbase + kk * 32, 16, 1024);
             const uint64_t b = smem_desc_sw128(vbase + kk * 2048, BK * 128, 1024);
-            umma_ss(tmem + 128, a, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            umma_ts(tmem + 128, pcol + kk * 8, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(bars.o_done + (j & 1));
           umma_commit(bars.v_empty + st);
@@ -340,15 +339,9 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         alive = false;
         break;
       }
-      // P row -> 128-byte-swizzled K-major tile: 16-byte chunk c of row `row`
-      // lands at chunk position (c ^ (row & 7)) of the row's 128-byte line.
-      uint8_t* prow = smem + L::OFF_P + sb * L::P_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
+      // P row -> TMEM lane `row`, columns [sb*64, sb*64 + 32) of the S buffer just read
+      tmem_st32(t_lane + sb * BK, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars.p_full + sb);
     }
