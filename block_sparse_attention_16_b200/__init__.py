@@ -26,7 +26,7 @@ __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
     "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait",
-    "lbsa_last_error", "lbsa_version", "library_path", "load_library",
+    "lbsa_select_head_noalloc", "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
 ]
@@ -83,6 +83,7 @@ def load_library():
         "lbsa_permute": (ctypes.c_int, [ctypes.POINTER(P), ctypes.POINTER(P), I32, P,
                                         ctypes.POINTER(_Desc), I32, P]),
         "lbsa_selftest_wait": (ctypes.c_int, [I64, P, P]),
+        "lbsa_select_head_noalloc": (ctypes.c_int, [P, I32, I32, I32, D, P, P, P, P]),
         "lbsa_last_error": (ctypes.c_char_p, []),
         "lbsa_version": (ctypes.c_int, []),
     }
@@ -282,6 +283,22 @@ def lbsa_selftest_wait(iters: int = 1000, stream=None) -> int:
     out = torch.zeros(1, dtype=torch.int32, device="cuda")
     _check(load_library().lbsa_selftest_wait(iters, _ptr(out), _stream(stream)))
     return int(out.item())
+
+
+def lbsa_select_head_noalloc(scores, p: float, counts=None, cols=None, status=None, stream=None):
+    """Head-scope selection into caller buffers; the library allocates nothing.
+
+    Returns (counts [B*H*nB], cols [B*H*nB*nB], status [1]) int32 device
+    tensors; row r's kept ids are cols[r*nB : r*nB + counts[r]].
+    """
+    B, H, nB, _ = scores.shape
+    dev = scores.device
+    counts = torch.empty(B * H * nB, dtype=torch.int32, device=dev) if counts is None else counts
+    cols = torch.empty(B * H * nB * nB, dtype=torch.int32, device=dev) if cols is None else cols
+    status = torch.empty(1, dtype=torch.int32, device=dev) if status is None else status
+    _check(load_library().lbsa_select_head_noalloc(_ptr(scores), B, H, nB, float(p), _ptr(counts), _ptr(cols),
+                                                   _ptr(status), _stream(stream)))
+    return counts, cols, status
 
 
 def lbsa_last_error() -> str:

@@ -401,6 +401,8 @@ int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream) {
 }  // extern "C"
 
 namespace lbsa {
+int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 namespace {
 // One thread waits on an mbarrier that nothing ever completes.
 __global__ void selftest_wait_kernel(long long iters, int32_t* out) {

@@ -80,4 +80,7 @@ cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, co
 
 cudaError_t launch_selftest_wait(long long iters, int32_t* out, cudaStream_t s);
 
+// Records `msg` as this thread's lbsa_last_error() text and returns `code`.
+int set_error(int code, const char* msg);
+
 }  // namespace lbsa

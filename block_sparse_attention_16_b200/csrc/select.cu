@@ -15,6 +15,9 @@
 // still reaches T.  Every element above tb is kept; of the elements equal to
 // tb (all of weight w(tb)), the ceil((T - S(tb+1)) / w(tb)) with the lowest
 // flat indices are kept.  This is exactly the sorted-prefix rule.
+#include <cstdio>
+#include <mutex>
+
 #include "lbsa_device.cuh"
 
 namespace lbsa {
@@ -474,3 +477,90 @@ cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blo
 }
 
 }  // namespace lbsa
+
+// ---------------------------------------------------------------- allocation-free head-scope selection
+// lbsa_select_head_noalloc runs the same head-scope kernels as lbsa_select,
+// but its scratch (radix histograms, per-head state, per-row tie counts) lives
+// in the file-scope device array below instead of memory obtained at run time,
+// and its outputs go to caller buffers.  The array is part of the loaded
+// module: every GPU that loads the library holds it until the process exits.
+namespace lbsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;   // 1 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in,
+// never a device address, so kernels are always given this pointer.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace lbsa
+
+extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t H, int32_t nB, double p,
+                                        int32_t* counts, int32_t* cols, int32_t* status, void* stream) {
+  using namespace lbsa;
+  if (!scores || (reinterpret_cast<uintptr_t>(scores) & 15u))
+    return set_error(LBSA_ERR_INVALID_ARG, "scores must be a non-NULL, 16-byte aligned device pointer");
+  if (!counts || !cols || !status) return set_error(LBSA_ERR_INVALID_ARG, "counts, cols and status must be non-NULL");
+  if (B < 1 || H < 1 || nB < 1) return set_error(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
+  if (!(p > 0.0) || !(p <= 1.0)) return set_error(LBSA_ERR_INVALID_ARG, "p must lie in (0, 1]");
+  const size_t need = select_head_workspace_bytes(B, H, nB);
+  if (need > kNoAllocScratchBytes) {
+    char msg[200];
+    std::snprintf(msg, sizeof(msg),
+                  "B*H=%d heads with nB=%d need %zu bytes of scratch; the static array holds %zu "
+                  "(B*H <= 64 with nB <= 1024 always fits)",
+                  B * H, nB, need, kNoAllocScratchBytes);
+    return set_error(LBSA_ERR_UNSUPPORTED, msg);
+  }
+  void* ws = nullptr;
+  cudaError_t e = noalloc_scratch(&ws);
+  if (e != cudaSuccess) return set_error(LBSA_ERR_CUDA, cudaGetErrorString(e));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = B * H;
+  const long long seg = static_cast<long long>(nB) * nB;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(ws);
+  HeadState* st = reinterpret_cast<HeadState*>(hist + static_cast<size_t>(G) * kBins);
+  int32_t* tie = reinterpret_cast<int32_t*>(st + G);
+  // the array keeps the previous call's contents: clear the histograms, the
+  // per-head state and the caller's status word before the passes
+  e = cudaMemsetAsync(ws, 0, static_cast<size_t>(G) * kBins * sizeof(unsigned long long) +
+                                 static_cast<size_t>(G) * sizeof(HeadState), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return set_error(LBSA_ERR_CUDA, cudaGetErrorString(e));
+  const uint32_t P = fixed_p(p);
+  const int keep_all = p >= 1.0 ? 1 : 0;
+  const int chunks = static_cast<int>(std::min<long long>(64, (seg + 4095) / 4096));
+  for (int pass = 0; pass < 3; ++pass) {
+    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
+    head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, status);
+  }
+  const long long rows = static_cast<long long>(G) * nB;
+  const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie);
+  head_tiescan_kernel<<<G, 1024, 0, s>>>(nB, st, tie);
+  head_emit_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie, counts, cols);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(LBSA_ERR_CUDA, cudaGetErrorString(e));
+  return LBSA_OK;
+}

@@ -200,6 +200,28 @@ int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const in
  * LBSA_ERR_TIMEOUT to *device_out (device int32).  Never hangs. */
 int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream);
 
+/* Head-scope selection that allocates nothing (the pages have no
+ * counterpart).  It serves callers that cannot call cudaMalloc: a host
+ * framework whose own caching allocator owns the device's memory (a
+ * cudaMalloc behind its back can fail once that pool has grown to the
+ * device's capacity), or a latency-bound serving loop that cannot accept the
+ * device-wide synchronisation a cudaMalloc may bring.  Same rule and results
+ * as lbsa_select(..., LBSA_SCOPE_HEAD, ...), written to caller buffers:
+ *   counts  device int32 [B*H*nB]: kept key blocks of row r = (b*H + h)*nB + i
+ *   cols    device int32 [B*H*nB*nB]: row r's ascending ids at cols[r*nB ...]
+ *   status  device int32 [1]: set to 0, then to the first device error
+ * Its scratch (radix histograms, per-head state, tie counts) lives in a
+ * 1 MiB file-scope device array that every GPU loading the library holds
+ * until the process exits; B*H <= 64 heads with nB <= 1024 always fit, larger
+ * sizes return LBSA_ERR_UNSUPPORTED with no launch.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress), so make
+ * that first call before any stream capture.  All calls on one GPU share that
+ * GPU's array and clear what they need at the start: calls that overlap on
+ * the same GPU (e.g. issued to different streams) race on it and must be
+ * serialised by the caller. */
+int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t H, int32_t nB, double p,
+                             int32_t* counts, int32_t* cols, int32_t* status, void* stream);
+
 /* Thread-local one-line reason for the last non-OK return of this thread. */
 const char* lbsa_last_error(void);
 
