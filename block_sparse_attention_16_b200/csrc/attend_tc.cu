@@ -293,12 +293,16 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_wait_ld();
       float x[64];
-      float mx = -INFINITY;
+      float mx8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         x[c] = (take && c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+        mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);      // 8 independent chains
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_new = fmaxf(m, mx);
       const bool need = (m != -INFINITY) && (m_new > m + 8.0f);
       if (m == -INFINITY) m = m_new;
@@ -324,17 +328,19 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           m = m_new;
         }
       }
-      float sum = 0.f;
+      float sum8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
       uint32_t pk[32];
       const float mref = (m == -INFINITY) ? 0.f : m;   // a row that has seen no key yet: all p = 0
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         const float p0 = ex2(x[2 * c] - mref);
         const float p1 = ex2(x[2 * c + 1] - mref);
-        sum += p0 + p1;
+        sum8[c & 7] += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
       }
-      l += sum;
+      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       if (s >= 2 && !mbar_wait(bars.o_done + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) {
         alive = false;
         break;

@@ -87,13 +87,13 @@ int make_tmap(CUtensorMap* map, const void* ptr, const lbsa_qkv_desc* d, int box
   return LBSA_OK;
 }
 
-// Per-device state: a status word for calls without a blockset and a
-// workspace that grows on demand (allocated outside the per-call path once it
-// is large enough).
+// Per-device state: a status word for calls without a blockset, and a memory
+// pool that serves blocksets and per-call scratch stream-ordered
+// (cudaMallocFromPoolAsync / cudaFreeAsync).  The pool keeps freed memory
+// cached, so after the first call of a given size nothing reaches the driver.
 struct DeviceState {
   int32_t* status = nullptr;
-  void* ws = nullptr;
-  size_t ws_bytes = 0;
+  cudaMemPool_t pool = nullptr;
 };
 std::mutex g_mu;
 DeviceState g_dev[64];
@@ -105,6 +105,17 @@ int device_state(DeviceState** out) {
   if (dev < 0 || dev >= 64) return fail(LBSA_ERR_UNSUPPORTED, "device %d", dev);
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState& s = g_dev[dev];
+  if (!s.pool) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    e = cudaMemPoolCreate(&s.pool, &props);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    cudaMemPoolSetAttribute(s.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  }
   if (!s.status) {
     e = cudaMalloc(&s.status, sizeof(int32_t));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(status)");
@@ -115,21 +126,23 @@ int device_state(DeviceState** out) {
   return LBSA_OK;
 }
 
-int workspace(DeviceState* s, size_t bytes, void** out) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (s->ws_bytes < bytes) {
-    if (s->ws) {
-      cudaError_t e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-      cudaFree(s->ws);
-      s->ws = nullptr;
-      s->ws_bytes = 0;
-    }
-    cudaError_t e = cudaMalloc(&s->ws, bytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
-    s->ws_bytes = bytes;
+// Stream-ordered scratch for one call: freed on the same stream after the
+// call's kernels, so concurrent calls on different streams never share it.
+struct Scratch {
+  void* ptr = nullptr;
+  cudaStream_t s = nullptr;
+  ~Scratch() {
+    if (ptr) cudaFreeAsync(ptr, s);
   }
-  *out = s->ws;
+};
+
+int scratch_alloc(DeviceState* ds, size_t bytes, cudaStream_t s, Scratch* out) {
+  cudaError_t e = cudaMallocFromPoolAsync(&out->ptr, bytes, ds->pool, s);
+  if (e != cudaSuccess) {
+    out->ptr = nullptr;
+    return cuda_fail(e, "cudaMallocFromPoolAsync(scratch)");
+  }
+  out->s = s;
   return LBSA_OK;
 }
 
@@ -141,8 +154,11 @@ int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStrea
   const size_t counts_bytes = ((R * sizeof(int32_t)) + 255) & ~size_t(255);
   const size_t bytes = counts_bytes + cols_bytes + 256;
   void* base = nullptr;
-  cudaError_t e = cudaMallocAsync(&base, bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(blockset)");
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LBSA_OK) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&base, bytes, ds->pool, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(blockset)");
   auto* bs = new lbsa_blockset;
   bs->B = B;
   bs->H = H;
@@ -189,20 +205,26 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
   DeviceState* ds = nullptr;
   if ((rc = device_state(&ds)) != LBSA_OK) return rc;
   cudaError_t e;
+  Scratch ws;
   if (mode == LBSA_SCORE_EXACT_MASS) {
-    lbsa::ScoreArgs a{desc->B, desc->H, desc->N_valid, desc->d, block, nB, scores, lse, ds->status, wait_limit()};
+    lbsa::ScoreArgs a{desc->B, desc->H, desc->N_valid, desc->d, block, nB, scores, lse, ds->status, wait_limit(),
+                      nullptr};
     if (desc->dtype == LBSA_BF16) {
       CUtensorMap tq, tk;
       if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
       if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
+      if ((rc = scratch_alloc(ds, lbsa::score_exact_bf16_workspace_bytes(desc->B, desc->H, desc->N_valid), s, &ws)) !=
+          LBSA_OK)
+        return rc;
+      a.scratch = static_cast<float*>(ws.ptr);
       e = lbsa::launch_score_exact_bf16(&tq, &tk, a, s);
     } else {
       e = lbsa::launch_score_exact_f32(static_cast<const float*>(q), static_cast<const float*>(k), *desc, a, s);
     }
   } else {
-    void* ws = nullptr;
-    if ((rc = workspace(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d), &ws)) != LBSA_OK) return rc;
-    e = lbsa::launch_meanpool(q, k, *desc, block, nB, scores, ws, s);
+    if ((rc = scratch_alloc(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d), s, &ws)) != LBSA_OK)
+      return rc;
+    e = lbsa::launch_meanpool(q, k, *desc, block, nB, scores, ws.ptr, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_score launch");
   return LBSA_OK;
@@ -228,12 +250,13 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
     e = lbsa::launch_select_row(scores, B * H * nB, nB, p, bs, s);
   } else {
     DeviceState* ds = nullptr;
-    void* ws = nullptr;
-    if ((rc = device_state(&ds)) != LBSA_OK || (rc = workspace(ds, lbsa::select_head_workspace_bytes(B, H, nB), &ws)) != LBSA_OK) {
+    Scratch ws;
+    if ((rc = device_state(&ds)) != LBSA_OK ||
+        (rc = scratch_alloc(ds, lbsa::select_head_workspace_bytes(B, H, nB), s, &ws)) != LBSA_OK) {
       lbsa_free(bs);
       return rc;
     }
-    e = lbsa::launch_select_head(scores, B, H, nB, p, bs, ws, s);
+    e = lbsa::launch_select_head(scores, B, H, nB, p, bs, ws.ptr, s);
   }
   if (e != cudaSuccess) {
     lbsa_free(bs);

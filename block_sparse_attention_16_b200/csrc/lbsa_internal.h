@@ -41,6 +41,7 @@ struct ScoreArgs {
   float* lse;
   int32_t* status;
   long long wait_limit;
+  float* scratch;       // bf16 exact mode: score_exact_bf16_workspace_bytes() of scratch
 };
 
 // bf16 tcgen05 kernels (attend_tc.cu, score_tc.cu)
@@ -48,6 +49,7 @@ cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, con
                                const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
                                     cudaStream_t s);
+size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid);
 
 // fp32 SIMT kernels (simt_f32.cu)
 cudaError_t launch_attend_f32(const float* q, const float* k, const float* v, const lbsa_qkv_desc& d,

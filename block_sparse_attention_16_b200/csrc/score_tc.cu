@@ -5,18 +5,23 @@
 // query block combine: the mean over the block's valid rows, so
 //   mass[b,h,i,j] = (1/|I_i|) sum_{r in I_i} sum_{c in J_j} softmax_c(q_r.k_c/sqrt(d)).
 //
-// One CTA owns a 128-row query tile and sweeps the whole key sequence twice in
-// 64-key steps: sweep 1 builds each row's log-sum-exp (online max / sum),
-// sweep 2 recomputes S = Q K^T, forms p = exp(s - lse) and sums it per row
-// over each 64-key chunk; warp shuffles reduce the chunk sums over the rows of
-// a warp, and the per-warp partials are combined in a fixed order at the end
-// (deterministic).  The row log-sum-exp stays in registers between sweeps, so
-// the kernel needs no memory beyond its inputs and outputs.
+// One sweep over the keys per 128-row query tile.  For every row and 64-key
+// chunk the softmax warps keep the online max m and sum l, and store the
+// chunk's log-sum-exp  L[r,c] = m + log2(sum_{k in chunk} 2^(x_k - m))  (base
+// 2, x = q.k * log2(e)/sqrt(d)) to a per-CTA scratch strip.  After the sweep
+// each row knows its lse, and  2^(L[r,c] - lse_r)  is the row's exact mass on
+// the chunk; warp shuffles sum it over the rows of a warp, and per-warp
+// partials are combined in a fixed order (deterministic).  Every Q K^T product
+// and every exponential of the dense pass is computed once.
 //
-// Warp roles (192 threads, two CTAs per SM): warps 0-3 softmax (thread t = tile
-// row t = TMEM lane t), warp 4 TMA producer (Q once, K 64-key tiles through a
-// ring), warp 5 UMMA issuer (S = Q K^T, M=128, N=64, K=d, double-buffered in
-// TMEM columns [0,64) and [64,128)).
+// Persistent grid (two CTAs per SM, each walking tiles with a grid stride), so
+// the scratch is bounded: gridDim.x * 128 * n_chunks floats.  Each thread
+// reads back only the scratch values it wrote itself.
+//
+// Warp roles (192 threads): warps 0-3 softmax (thread t = tile row t = TMEM
+// lane t), warp 4 TMA producer (Q per tile, K 64-key tiles through a ring),
+// warp 5 UMMA issuer (S = Q K^T, M=128, N=64, K=d, double-buffered in TMEM
+// columns [0,64) and [64,128)).
 #include "lbsa_device.cuh"
 
 namespace lbsa {
@@ -27,6 +32,7 @@ constexpr int BK = 64;
 constexpr int NS = 3;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 128;
+constexpr int kCtasPerSm = 2;
 
 template <int D>
 struct Layout {
@@ -35,33 +41,46 @@ struct Layout {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_BAR = OFF_K + NS * K_BYTES;
-  // q_full, k_full[NS], k_empty[NS], s_full[2], s_free[2], drain
-  static constexpr int NBAR = 1 + 2 * NS + 5;
+  // q_full, q_empty, k_full[NS], k_empty[NS], s_full[2], s_free[2], drain
+  static constexpr int NBAR = 2 + 2 * NS + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_PART = OFF_MISC + 16;
   static size_t bytes(int n_chunks) { return OFF_PART + static_cast<size_t>(4) * n_chunks * 4 + 1024; }
 };
 
+struct TileIdx {
+  int tile, h, bb;
+};
+__device__ __forceinline__ TileIdx tile_of(int g, int tiles_per_bh, int H) {
+  TileIdx t;
+  t.tile = g % tiles_per_bh;
+  const int bh = g / tiles_per_bh;
+  t.h = bh % H;
+  t.bb = bh / H;
+  return t;
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const ScoreArgs args, float scale_log2) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
   const int N = args.N_valid;
   const int n_chunks = (N + BK - 1) / BK;
-  const int n_steps = 2 * n_chunks;
+  const int tiles_per_bh = (N + BM - 1) / BM;
+  const int total_tiles = tiles_per_bh * args.H * args.B;
   const long long wl = args.wait_limit;
   if (*reinterpret_cast<volatile int32_t*>(args.status) == LBSA_ERR_TIMEOUT) return;
 
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bar;
-  uint64_t* k_full = bar + 1;
-  uint64_t* k_empty = bar + 1 + NS;
-  uint64_t* s_full = bar + 1 + 2 * NS;
+  uint64_t* q_empty = bar + 1;
+  uint64_t* k_full = bar + 2;
+  uint64_t* k_empty = bar + 2 + NS;
+  uint64_t* s_full = bar + 2 + 2 * NS;
   uint64_t* s_free = s_full + 2;
   uint64_t* drain = s_free + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -70,6 +89,7 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
 
   if (tid == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < NS; ++i) {
       mbar_init(k_full + i, 1);
       mbar_init(k_empty + i, 1);
@@ -92,113 +112,143 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
   const uint32_t tmem = misc[0];
 
   if (warp == 4) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmap_q);
       prefetch_tmap(&tmap_k);
       uint8_t* sQ = smem + L::OFF_Q;
-      mbar_arrive_expect_tx(q_full, L::Q_BYTES);
-      for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, q_full, c * 64, tile * BM, h, bb);
-      int issued = 0;
-      for (int s = 0; s < n_steps; ++s) {
-        const int st = s % NS;
-        if (s >= NS && !mbar_wait(k_empty + st, ((s / NS) & 1) ^ 1, wl, args.status, abort_flag)) break;
-        const int key0 = (s % n_chunks) * BK;
-        uint8_t* sK = smem + L::OFF_K + st * L::K_BYTES;
-        mbar_arrive_expect_tx(k_full + st, L::K_BYTES);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, key0, h, bb);
-        issued = s + 1;
+      long long s = 0;       // global step counter (ring position)
+      int it = 0;            // tiles handled by this CTA
+      bool ok = true;
+      for (int g = blockIdx.x; ok && g < total_tiles; g += gridDim.x, ++it) {
+        const TileIdx t = tile_of(g, tiles_per_bh, args.H);
+        if (it >= 1 && !mbar_wait(q_empty, (it - 1) & 1, wl, args.status, abort_flag)) break;
+        mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+        for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, q_full, c * 64, t.tile * BM, t.h, t.bb);
+        for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+          const int st = static_cast<int>(s % NS);
+          if (s >= NS && !mbar_wait(k_empty + st, static_cast<uint32_t>((s / NS) & 1) ^ 1u, wl, args.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sK = smem + L::OFF_K + st * L::K_BYTES;
+          mbar_arrive_expect_tx(k_full + st, L::K_BYTES);
+          for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, ch * BK, t.h, t.bb);
+        }
       }
       if (*abort_flag) {
-        mbar_wait(q_full, 0, wl, args.status, nullptr);
-        for (int s = (issued > NS ? issued - NS : 0); s < issued; ++s)
-          mbar_wait(k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
+        // let copies still in flight land before the CTA can exit
+        for (long long r = (s > NS ? s - NS : 0); r < s; ++r)
+          mbar_wait(k_full + r % NS, static_cast<uint32_t>((r / NS) & 1), wl, args.status, nullptr);
       }
     }
   } else if (warp == 5) {
+    // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(BM, BK, 0);
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK0 = smem_u32(smem + L::OFF_K);
-      bool ok = mbar_wait(q_full, 0, wl, args.status, abort_flag);
-      for (int s = 0; ok && s < n_steps; ++s) {
-        const int st = s % NS;
-        const int sb = s & 1;
-        if (!mbar_wait(k_full + st, (s / NS) & 1, wl, args.status, abort_flag)) break;
-        if (s >= 2 && !mbar_wait(s_free + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t kbase = sK0 + st * L::K_BYTES;
+      long long s = 0;
+      int it = 0;
+      bool ok = true;
+      for (int g = blockIdx.x; ok && g < total_tiles; g += gridDim.x, ++it) {
+        if (!mbar_wait(q_full, it & 1, wl, args.status, abort_flag)) break;
+        for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+          const int st = static_cast<int>(s % NS);
+          const int sb = static_cast<int>(s & 1);
+          if (!mbar_wait(k_full + st, static_cast<uint32_t>((s / NS) & 1), wl, args.status, abort_flag) ||
+              (s >= 2 && !mbar_wait(s_free + sb, static_cast<uint32_t>(((s - 2) >> 1) & 1), wl, args.status, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kbase = sK0 + st * L::K_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * (BM * 128) + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * (BK * 128) + off, 16, 1024);
-          umma_ss(tmem + sb * BK, a, b, idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk & 3) * 32;
+            const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * (BM * 128) + off, 16, 1024);
+            const uint64_t b = smem_desc_sw128(kbase + (kk >> 2) * (BK * 128) + off, 16, 1024);
+            umma_ss(tmem + sb * BK, a, b, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(s_full + sb);
+          umma_commit(k_empty + st);
         }
-        umma_commit(s_full + sb);
-        umma_commit(k_empty + st);
+        umma_commit(q_empty);          // Q may be replaced once this tile's UMMAs are done
       }
       umma_commit(drain);
       mbar_wait(drain, 0, wl, args.status, nullptr);
     }
   } else {
+    // ------------------------------------------------------------ softmax (warps 0-3)
     const int row = tid;
-    const int grow = tile * BM + row;
-    const bool valid_row = grow < N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m = -INFINITY, l = 0.f, lse2 = 0.f;
-    for (int s = 0; s < n_steps; ++s) {
-      const int sb = s & 1;
-      if (!mbar_wait(s_full + sb, (s >> 1) & 1, wl, args.status, abort_flag)) break;
-      tc_fence_after();
-      uint32_t r[64];
-      tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free + sb);
-      const int chunk = s % n_chunks;
-      const int nvk = N - chunk * BK;
-      if (s < n_chunks) {
+    float* strip = args.scratch + static_cast<long long>(blockIdx.x) * n_chunks * BM;   // [n_chunks][128]
+    long long s = 0;
+    bool alive = true;
+    for (int g = blockIdx.x; alive && g < total_tiles; g += gridDim.x) {
+      const TileIdx t = tile_of(g, tiles_per_bh, args.H);
+      const int grow = t.tile * BM + row;
+      const bool valid_row = grow < N;
+      float m = -INFINITY, l = 0.f;
+      for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+        const int sb = static_cast<int>(s & 1);
+        if (!mbar_wait(s_full + sb, static_cast<uint32_t>((s >> 1) & 1), wl, args.status, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(s_free + sb);
+        const int nvk = N - ch * BK;
         float x[64];
-        float mx = -INFINITY;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           x[c] = (c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
+          acc[c & 7] = fmaxf(acc[c & 7], x[c]);      // 8 independent chains
         }
-        const float m_new = fmaxf(m, mx);
-        float acc = (m == -INFINITY) ? 0.f : l * ex2(m - m_new);
+        const float mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                               fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
+        const float m_new = fmaxf(m, mx);    // finite: every chunk holds a valid key
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc += ex2(x[c] - m_new);
-        l = acc;
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c & 7] += ex2(x[c] - m_new);
+        const float bsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        l = (m == -INFINITY) ? bsum : fmaf(l, ex2(m - m_new), bsum);
         m = m_new;
-        if (s == n_chunks - 1) lse2 = m + __log2f(l);
-      } else {
-        float rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          rs += (c < nvk) ? ex2(__uint_as_float(r[c]) * scale_log2 - lse2) : 0.f;
-        if (!valid_row) rs = 0.f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
-        if (lane == 0) part[warp * n_chunks + chunk] = rs;
+        strip[static_cast<long long>(ch) * BM + row] = m + __log2f(bsum);
       }
-    }
-    named_bar_sync(1, 128);
-    if (!*abort_flag) {
+      if (!alive) break;
+      const float lse2 = m + __log2f(l);
+      // mass of each chunk, summed over this warp's rows
+      for (int ch = 0; ch < n_chunks; ++ch) {
+        float v = valid_row ? ex2(strip[static_cast<long long>(ch) * BM + row] - lse2) : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) part[warp * n_chunks + ch] = v;
+      }
+      named_bar_sync(1, 128);
       const int nB = args.nB;
-      const long long hrow = (static_cast<long long>(bb) * args.H + h) * nB;
+      const long long hrow = (static_cast<long long>(t.bb) * args.H + t.h) * nB;
       if (args.block == 64) {
         for (int o = tid; o < 2 * nB; o += 128) {
           const int half = o / nB, kb = o % nB;
-          const int qb = 2 * tile + half;
+          const int qb = 2 * t.tile + half;
           if (qb >= nB) continue;
           const int rv = min(64, N - qb * 64);
-          const float v = (part[(2 * half) * n_chunks + kb] + part[(2 * half + 1) * n_chunks + kb]) / static_cast<float>(rv);
+          const float v = (part[(2 * half) * n_chunks + kb] + part[(2 * half + 1) * n_chunks + kb]) /
+                          static_cast<float>(rv);
           args.scores[(hrow + qb) * nB + kb] = v;
         }
       } else {
-        const int qb = tile;
+        const int qb = t.tile;
         const int rv = min(128, N - qb * 128);
         for (int kb = tid; kb < nB; kb += 128) {
           float v = 0.f;
@@ -211,7 +261,8 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
         }
       }
       if (args.lse && valid_row)
-        args.lse[(static_cast<long long>(bb) * args.H + h) * N + grow] = lse2 * 0.69314718055994531f;
+        args.lse[(static_cast<long long>(t.bb) * args.H + t.h) * N + grow] = lse2 * 0.69314718055994531f;
+      named_bar_sync(1, 128);           // part[] is reused by the next tile
     }
   }
   tc_fence_before();
@@ -222,13 +273,34 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
   }
 }
 
+int g_num_sms = 0;
+
+int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+int score_grid(int N, int H, int B) {
+  const long long tiles = static_cast<long long>((N + BM - 1) / BM) * H * B;
+  return static_cast<int>(std::min<long long>(tiles, static_cast<long long>(kCtasPerSm) * num_sms()));
+}
+
 }  // namespace
+
+size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid) {
+  const int n_chunks = (N_valid + BK - 1) / BK;
+  return static_cast<size_t>(score_grid(N_valid, H, B)) * BM * n_chunks * sizeof(float) + 256;
+}
 
 cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
                                     cudaStream_t s) {
-  const int tiles = (a.N_valid + BM - 1) / BM;
   const int n_chunks = (a.N_valid + BK - 1) / BK;
-  dim3 grid(tiles, a.H, a.B);
+  dim3 grid(score_grid(a.N_valid, a.H, a.B));
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
   if (a.d == 128) {
     const size_t smem = Layout<128>::bytes(n_chunks);
