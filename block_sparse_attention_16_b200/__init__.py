@@ -54,7 +54,8 @@ _LIB = None
 
 
 def library_path() -> str:
-    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbsa.so")
+    """The in-tree liblbsa.so, or the file named by the LBSA_LIBRARY environment variable."""
+    return os.environ.get("LBSA_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblbsa.so")
 
 
 def load_library():

@@ -29,7 +29,21 @@ def _headers_mtime():
     return max(os.path.getmtime(h) for h in hs)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, defines=(), out: str | None = None,
+          obj_dir: str | None = None) -> str:
+    """Build liblbsa.so; `defines` (e.g. ["LBSA_SCORE_POLY_EVERY=4"]) and `out` /
+    `obj_dir` build a variant library elsewhere."""
+    global OUT, OBJ
+    out_path, obj_path = out or OUT, obj_dir or OBJ
+    saved = OUT, OBJ
+    OUT, OBJ = out_path, obj_path
+    try:
+        return _build(force, verbose, [f"-D{d}" for d in defines])
+    finally:
+        OUT, OBJ = saved
+
+
+def _build(force, verbose, dflags) -> str:
     os.makedirs(OBJ, exist_ok=True)
     srcs = sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
     hdr = _headers_mtime()
@@ -39,7 +53,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         obj = os.path.join(OBJ, f[:-3] + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr):
-            cmd = [NVCC, *FLAGS, "-c", src, "-o", obj]
+            cmd = [NVCC, *FLAGS, *dflags, "-c", src, "-o", obj]
             if verbose:
                 print(" ".join(cmd), flush=True)
             subprocess.run(cmd, check=True)

@@ -37,7 +37,6 @@ constexpr int kThreads = 192;
 constexpr int kMaxBlocks = 4096;  // nB bound (bitmap size)
 constexpr int kMaxWords = kMaxBlocks / 32;
 constexpr uint32_t kTmemCols = 256;
-
 template <int D>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
@@ -286,23 +285,26 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       tc_fence_after();
       const uint32_t e = sched[s / spb];
       const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
-      const bool take = ((e >> 30) >> half) & 1u;
       const int nvk = args.N_valid - key0;     // valid keys in this step (may exceed 64)
+      // warp-uniform: rows 0-63 (warps 0,1) and 64-127 (warps 2,3) are the two halves
+      const bool take = (((e >> 30) >> half) & 1u) && nvk > 0;
+      const bool full = take && nvk >= 64;
       uint32_t r[64];
       tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_wait_ld();
-      float x[64];
-      float mx8[8];
+      // row max of the raw logits (the scale is positive), 4 independent chains
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (full) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+        for (int c = 0; c < 64; c += 2)
+          mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+      } else if (take) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = (take && c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
-        mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);      // 8 independent chains
+        for (int c = 0; c < 64; ++c)
+          if (c < nvk) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(r[c]));
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
       const float m_new = fmaxf(m, mx);
       const bool need = (m != -INFINITY) && (m_new > m + 8.0f);
       if (m == -INFINITY) m = m_new;
@@ -328,18 +330,37 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
           m = m_new;
         }
       }
+      // p = 2^(s*scale - m): one packed FMA per pair, MUFU ex2, packed row-sum adds
+      uint32_t pk[32];
+      unsigned long long sum4[4] = {0ull, 0ull, 0ull, 0ull};
+      const unsigned long long sc2 = f2_as_u64(scale_log2, scale_log2);
+      const unsigned long long nm2 = f2_as_u64(-m, -m);
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float v0, v1;
+          u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
+          const float p0 = ex2(v0), p1 = ex2(v1);
+          sum4[c & 3] = fadd2(sum4[c & 3], f2_as_u64(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+      } else if (take) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float v0, v1;
+          u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
+          const float p0 = (2 * c < nvk) ? ex2(v0) : 0.f;
+          const float p1 = (2 * c + 1 < nvk) ? ex2(v1) : 0.f;
+          sum4[c & 3] = fadd2(sum4[c & 3], f2_as_u64(p0, p1));
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
       float sum8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sum8[i] = 0.f;
-      uint32_t pk[32];
-      const float mref = (m == -INFINITY) ? 0.f : m;   // a row that has seen no key yet: all p = 0
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2(x[2 * c] - mref);
-        const float p1 = ex2(x[2 * c + 1] - mref);
-        sum8[c & 7] += p0 + p1;
-        pk[c] = pack_bf16x2(p0, p1);
-      }
+      for (int i = 0; i < 4; ++i) u64_as_f2(sum4[i], sum8[2 * i], sum8[2 * i + 1]);
       l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       if (s >= 2 && !mbar_wait(bars.o_done + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) {
         alive = false;

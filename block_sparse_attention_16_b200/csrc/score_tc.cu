@@ -33,7 +33,6 @@ constexpr int NS = 3;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 128;
 constexpr int kCtasPerSm = 2;
-
 template <int D>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
@@ -204,23 +203,41 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
         tc_fence_before();
         mbar_arrive(s_free + sb);
         const int nvk = N - ch * BK;
-        float x[64];
-        float acc[8];
+        // row max of the raw logits (the scale is positive), 4 independent chains
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (nvk >= 64) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = -INFINITY;
+          for (int c = 0; c < 64; c += 2)
+            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+        } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] = (c < nvk) ? __uint_as_float(r[c]) * scale_log2 : -INFINITY;
-          acc[c & 7] = fmaxf(acc[c & 7], x[c]);      // 8 independent chains
+          for (int c = 0; c < 64; ++c)
+            if (c < nvk) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(r[c]));
         }
-        const float mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
-                               fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
-        const float m_new = fmaxf(m, mx);    // finite: every chunk holds a valid key
+        const float m_new = fmaxf(m, fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2);
+        // sum of 2^(s*scale - m_new): packed FMA per pair, MUFU ex2, packed adds
+        const unsigned long long sc2 = f2_as_u64(scale_log2, scale_log2);
+        const unsigned long long nm2 = f2_as_u64(-m_new, -m_new);
+        unsigned long long acc4[4] = {0ull, 0ull, 0ull, 0ull};
+        if (nvk >= 64) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+          for (int c = 0; c < 32; ++c) {
+            float v0, v1;
+            u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
+            acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(ex2(v0), ex2(v1)));
+          }
+        } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c & 7] += ex2(x[c] - m_new);
-        const float bsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          for (int c = 0; c < 32; ++c) {
+            float v0, v1;
+            u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
+            acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(2 * c < nvk ? ex2(v0) : 0.f, 2 * c + 1 < nvk ? ex2(v1) : 0.f));
+          }
+        }
+        float a8[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) u64_as_f2(acc4[i], a8[2 * i], a8[2 * i + 1]);
+        const float bsum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
         l = (m == -INFINITY) ? bsum : fmaf(l, ex2(m - m_new), bsum);
         m = m_new;
         strip[static_cast<long long>(ch) * BM + row] = m + __log2f(bsum);
