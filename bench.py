@@ -203,12 +203,11 @@ def run_own(args, rank, world):
     from block_sparse_attention_16_b200.build import build
     from block_sparse_attention_16_b200.workload import get_workload, make_qkv
 
-    if rank == 0:
-        build()
-    if world > 1:
-        torch.distributed.barrier()
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
+    if rank == 0:
+        build()
+    barrier(dev)
     lbsa.load_library()
     wl = get_workload(WORKLOAD)
     T, H, W = wl.grid
@@ -252,8 +251,7 @@ def run_own(args, rank, world):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = Clocks(dev.index, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
                     if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/lbsa_clocks_{rank}.csv")
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(dev)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -262,14 +260,9 @@ def run_own(args, rank, world):
         o, bs = step(evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    barrier(dev)
     clk = clocks.stop()
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     stage_names = ["permute", "score", "select", "attend", "unpermute"]
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(stage_names)}
     ms_per_step = total_ms / args.steps
@@ -315,11 +308,7 @@ def run_own(args, rank, world):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     bytes_in = 3 * q.numel() * q.element_size()
     bytes_out = q.numel() * q.element_size()
 

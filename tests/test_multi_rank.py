@@ -1,0 +1,72 @@
+"""World-size-2 gloo tests (CPU) of the multi-rank host logic."""
+import itertools
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from block_sparse_attention_16_b200.multi import lpt_shards, max_over_ranks, shard_loads, barrier
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, weights, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        shards = lpt_shards(weights, world)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, shards)
+        assert all(g == shards for g in gathered), "ranks disagree on the split"
+        mine = shards[rank]
+        t = 10.0 + 5.0 * rank + 0.25 * len(mine)
+        tmax = max_over_ranks(t)
+        barrier()
+        with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+            f.write(f"{tmax} {','.join(map(str, mine))}\n")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_and_reduce(tmp_path):
+    rng = np.random.default_rng(0)
+    weights = (rng.random(12) * 100).round(3).tolist()       # kept pairs per (batch, head)
+    port = _free_port()
+    mp.start_processes(_worker, args=(2, port, weights, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    lines = [open(tmp_path / f"rank{r}.txt").read().split() for r in range(2)]
+    shards = lpt_shards(weights, 2)
+    expect_max = max(10.0 + 5.0 * r + 0.25 * len(shards[r]) for r in range(2))
+    for r, (tmax, mine) in enumerate(lines):
+        assert float(tmax) == expect_max
+        assert list(map(int, mine.split(","))) == shards[r]
+
+
+def test_lpt_is_a_partition_and_within_four_thirds_of_optimal():
+    rng = np.random.default_rng(1)
+    for trial in range(40):
+        n = int(rng.integers(1, 11))
+        world = int(rng.integers(1, 4))
+        w = rng.integers(1, 50, size=n).tolist()
+        shards = lpt_shards(w, world)
+        assert sorted(i for s in shards for i in s) == list(range(n))
+        best = min(max(sum(w[i] for i in range(n) if a[i] == r) for r in range(world))
+                   for a in itertools.product(range(world), repeat=n))
+        assert max(shard_loads(w, shards)) <= (4 / 3 - 1 / (3 * world)) * best + 1e-9
+
+
+def test_single_process_helpers_are_identity():
+    assert max_over_ranks(3.5) == 3.5
+    assert lpt_shards([5, 5, 5], 1) == [[0, 1, 2]]
+    with pytest.raises(ValueError):
+        lpt_shards([1], 0)
