@@ -344,43 +344,19 @@ def run_own(args, rank, world):
 
 
 def load_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it covers this kernel version."""
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's sources changed since those counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path))
-    return d.get(kernel)
-
-
-def run_profile(kernel):
-    """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
-    than L2), one warm-up pass of the path, then two launches of `kernel`."""
-    import dataclasses
-
-    import block_sparse_attention_16_b200 as lbsa
-    from block_sparse_attention_16_b200.build import build
-    from block_sparse_attention_16_b200.workload import get_workload, make_qkv
-
-    build()
-    wl = dataclasses.replace(get_workload(WORKLOAD), H=6)
-    T, H, W = wl.grid
-    q, k, v = make_qkv(wl, device="cuda")
-    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4), device="cuda")
-    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
-    scores = lbsa.lbsa_score(qp, kp, wl.block)
-    bs = lbsa.lbsa_select(scores, wl.block, P, "row")
-    lbsa.lbsa_attend(qp, kp, vp, bs)
-    for _ in range(2):
-        if kernel == "attend":
-            lbsa.lbsa_attend(qp, kp, vp, bs)
-        elif kernel == "score":
-            lbsa.lbsa_score(qp, kp, wl.block, scores=scores)
-        elif kernel == "select":
-            lbsa.lbsa_select(scores, wl.block, P, "row")
-    torch.cuda.synchronize()
-    assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
-    print(f"profile case {kernel}: ok")
-    return 0
+    d = json.load(open(path)).get(kernel)
+    if not d:
+        return None
+    h = hashlib.sha256()
+    for f in d["files"]:
+        h.update(open(os.path.join(ROOT, "block_sparse_attention_16_b200", "csrc", f), "rb").read())
+    return d["bytes"] if h.hexdigest()[:16] == d["source_hash"] else None
 
 
 def main():
