@@ -201,6 +201,7 @@ def config_dict(wl, world):
 def run_own(args, rank, world):
     import block_sparse_attention_16_b200 as lbsa
     from block_sparse_attention_16_b200.build import build
+    from block_sparse_attention_16_b200.multi import barrier, max_over_ranks
     from block_sparse_attention_16_b200.workload import get_workload, make_qkv
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
