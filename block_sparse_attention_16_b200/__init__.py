@@ -280,9 +280,10 @@ def lbsa_permute(xs, perm, inverse: bool = False, outs=None, stream=None):
     return outs
 
 
-def lbsa_selftest_wait(iters: int = 1000, stream=None) -> int:
+def lbsa_selftest_wait(limit_us: int = 1000, stream=None) -> int:
+    """Run the bounded-wait self test; returns the device status it reported."""
     out = torch.zeros(1, dtype=torch.int32, device="cuda")
-    _check(load_library().lbsa_selftest_wait(iters, _ptr(out), _stream(stream)))
+    _check(load_library().lbsa_selftest_wait(limit_us, _ptr(out), _stream(stream)))
     return int(out.item())
 
 

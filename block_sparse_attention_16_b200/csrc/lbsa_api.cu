@@ -413,10 +413,10 @@ int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const in
   return LBSA_OK;
 }
 
-int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream) {
+int lbsa_selftest_wait(int64_t limit_us, int32_t* device_out, void* stream) {
   if (!device_out) return fail(LBSA_ERR_INVALID_ARG, "device_out is NULL");
-  if (iters < 1 || iters > (1ll << 30)) return fail(LBSA_ERR_INVALID_ARG, "iters out of range");
-  cudaError_t e = lbsa::launch_selftest_wait(iters, device_out, static_cast<cudaStream_t>(stream));
+  if (limit_us < 1 || limit_us > 10000000) return fail(LBSA_ERR_INVALID_ARG, "limit_us must lie in [1, 1e7]");
+  cudaError_t e = lbsa::launch_selftest_wait(limit_us * 1000, device_out, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_selftest_wait launch");
   return LBSA_OK;
 }
@@ -428,7 +428,7 @@ int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
 
 namespace {
 // One thread waits on an mbarrier that nothing ever completes.
-__global__ void selftest_wait_kernel(long long iters, int32_t* out) {
+__global__ void selftest_wait_kernel(long long limit_ns, int32_t* out) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   __shared__ int32_t st;
@@ -440,14 +440,14 @@ __global__ void selftest_wait_kernel(long long iters, int32_t* out) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const bool ok = mbar_wait(&bar, 0, iters, &st, &abort_flag);
+    const bool ok = mbar_wait(&bar, 0, limit_ns, &st, &abort_flag);
     *out = ok ? LBSA_OK : st;
   }
 }
 }  // namespace
 
-cudaError_t launch_selftest_wait(long long iters, int32_t* out, cudaStream_t s) {
-  selftest_wait_kernel<<<1, 32, 0, s>>>(iters, out);
+cudaError_t launch_selftest_wait(long long limit_ns, int32_t* out, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, out);
   return cudaGetLastError();
 }
 }  // namespace lbsa

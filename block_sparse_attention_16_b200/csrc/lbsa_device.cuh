@@ -38,27 +38,53 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// Suspend-time hint (ns) for try_wait: a waiting thread sleeps until the phase
+// completes or the hint runs out, instead of spinning on issue slots that the
+// working warps of the SM need.
+#ifndef LBSA_WAIT_HINT_NS
+#define LBSA_WAIT_HINT_NS 0
+#endif
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
+  if (LBSA_WAIT_HINT_NS > 0) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(LBSA_WAIT_HINT_NS))
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+  }
   return ok != 0;
 }
 
-// Bounded wait for the phase with the given parity.  Each try_wait suspends
-// for a hardware time slice, so `limit` polls bound the wait to well under a
-// few seconds.  On expiry: record LBSA_ERR_TIMEOUT, set the CTA's abort flag
-// and return false; callers then leave their loops.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit,
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for the phase with the given parity, at most `limit_ns`
+// nanoseconds of wall time (%globaltimer).  On expiry: record
+// LBSA_ERR_TIMEOUT, set the CTA's abort flag and return false; callers then
+// leave their loops.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit_ns,
                                           int32_t* status, volatile int* abort_flag) {
-  for (long long it = 0; it < limit; ++it) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort_flag && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > static_cast<uint64_t>(limit_ns)) break;
   }
   raise_status(status, LBSA_ERR_TIMEOUT);
   if (abort_flag) *abort_flag = 1;

@@ -5,7 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/lbsa.h"
+#include "lbsa.h"   // include/ is on the include path
 
 // Library-owned selection result.  Row r = (b*H + h)*nB + i owns the slot
 // cols[r*nB .. r*nB + nB); counts[r] entries of it are valid, ascending.
@@ -22,7 +22,7 @@ struct lbsa_blockset {
 
 namespace lbsa {
 
-constexpr long long kDefaultWaitLimit = 1ll << 20;   // mbarrier polls before a wait gives up (~1 s)
+constexpr long long kDefaultWaitLimit = 2000000000ll;   // ns a device wait may take before it gives up (2 s)
 
 struct AttendArgs {
   int B, H, N_valid, d, block, nB;
@@ -80,7 +80,7 @@ cudaError_t launch_partition_perm(int T, int Hg, int Wg, int kind, int tt, int t
 cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, const int32_t* perm,
                            const lbsa_qkv_desc& d, int inverse, cudaStream_t s);
 
-cudaError_t launch_selftest_wait(long long iters, int32_t* out, cudaStream_t s);
+cudaError_t launch_selftest_wait(long long limit_ns, int32_t* out, cudaStream_t s);
 
 // Records `msg` as this thread's lbsa_last_error() text and returns `code`.
 int set_error(int code, const char* msg);

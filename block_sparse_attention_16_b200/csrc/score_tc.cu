@@ -244,12 +244,21 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
       }
       if (!alive) break;
       const float lse2 = m + __log2f(l);
-      // mass of each chunk, summed over this warp's rows
-      for (int ch = 0; ch < n_chunks; ++ch) {
-        float v = valid_row ? ex2(strip[static_cast<long long>(ch) * BM + row] - lse2) : 0.f;
+      // mass of each chunk, summed over this warp's rows.  The strip is read
+      // back 16 chunks at a time so that 16 loads are in flight per thread.
+      for (int ch0 = 0; ch0 < n_chunks; ch0 += 16) {
+        float Lv[16];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) part[warp * n_chunks + ch] = v;
+        for (int u = 0; u < 16; ++u)
+          Lv[u] = (ch0 + u < n_chunks) ? strip[static_cast<long long>(ch0 + u) * BM + row] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (ch0 + u >= n_chunks) break;
+          float v = valid_row ? ex2(Lv[u] - lse2) : 0.f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if (lane == 0) part[warp * n_chunks + ch0 + u] = v;
+        }
       }
       named_bar_sync(1, 128);
       const int nB = args.nB;

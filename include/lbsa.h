@@ -196,9 +196,10 @@ int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const in
                  const lbsa_qkv_desc* desc, int32_t inverse, void* stream);
 
 /* Self-test of the bounded-wait machinery: one kernel waits on an mbarrier
- * that nothing completes, gives up after `iters` polls and writes
- * LBSA_ERR_TIMEOUT to *device_out (device int32).  Never hangs. */
-int lbsa_selftest_wait(int64_t iters, int32_t* device_out, void* stream);
+ * that nothing completes, gives up after `limit_us` microseconds of wall time
+ * (the same check every device wait of the library makes, with a 2 s limit)
+ * and writes LBSA_ERR_TIMEOUT to *device_out (device int32).  Never hangs. */
+int lbsa_selftest_wait(int64_t limit_us, int32_t* device_out, void* stream);
 
 /* Head-scope selection that allocates nothing (the pages have no
  * counterpart).  It serves callers that cannot call cudaMalloc: a host
