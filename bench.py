@@ -360,6 +360,199 @@ def load_traffic(kernel):
     return d["bytes"] if h.hexdigest()[:16] == d["source_hash"] else None
 
 
+def run_profile(kernel):
+    """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
+    than L2), one warm-up pass of the path, then two launches of `kernel`."""
+    import dataclasses
+
+    import block_sparse_attention_16_b200 as lbsa
+    from block_sparse_attention_16_b200.build import build
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv
+
+    build()
+    wl = dataclasses.replace(get_workload(WORKLOAD), H=6)
+    T, H, W = wl.grid
+    q, k, v = make_qkv(wl, device="cuda")
+    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4), device="cuda")
+    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+    scores = lbsa.lbsa_score(qp, kp, wl.block)
+    bs = lbsa.lbsa_select(scores, wl.block, P, "row")
+    lbsa.lbsa_attend(qp, kp, vp, bs)
+    for _ in range(2):
+        if kernel == "attend":
+            lbsa.lbsa_attend(qp, kp, vp, bs)
+        elif kernel == "score":
+            lbsa.lbsa_score(qp, kp, wl.block, scores=scores)
+        elif kernel == "select":
+            lbsa.lbsa_select(scores, wl.block, P, "row")
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+    print(f"profile case {kernel}: ok")
+    return 0
+
+
+def _timer(fn, n=10, warm=3, flush=None):
+    """Median device time (ms) of fn() over n runs, CUDA events on the current stream."""
+    for _ in range(warm):
+        fn()
+    ts = []
+    for _ in range(n):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return {"median": ts[len(ts) // 2], "p10": ts[max(0, len(ts) // 10)], "p90": ts[min(len(ts) - 1, (9 * len(ts)) // 10)]}
+
+
+def run_sweep(args):
+    """Per-stage timings on every workload (one JSON line per measurement)."""
+    import block_sparse_attention_16_b200 as lbsa
+    from block_sparse_attention_16_b200.build import build
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv, make_qkv_f32, redraw_qkv
+
+    build()
+    torch.cuda.set_device(0)
+    pk = peaks()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")   # 256 MB L2 flush
+    out = []
+
+    def emit(**kw):
+        line = json.dumps(kw)
+        out.append(line)
+        print(line, flush=True)
+
+    def flops_of(bs, wl):
+        rp, col = lbsa.lbsa_blockset_export(bs)
+        rp, col = rp.cpu().numpy(), col.cpu().numpy()
+        m = kept_mask(rp, col, wl.B * wl.H * wl.n_blocks, wl.n_blocks).reshape(wl.B * wl.H, wl.n_blocks, wl.n_blocks)
+        return attention_flops(m, wl.n_blocks, wl.block, wl.n_valid, wl.d), m
+
+    def hbm(nbytes, ms):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"GB/s": gbs, "frac_hbm": gbs / pk["hbm_gbs"]}
+
+    def tfl(fl, ms):
+        t = fl / (ms * 1e-3) / 1e12
+        return {"TFLOP/s": t, "frac_bf16_sustained": t / pk["bf16_sustained"], "frac_bf16_burst": t / pk["bf16"]}
+
+    # tiny fp32 workload (true-fp32 SIMT kernels)
+    wl = get_workload("tiny")
+    q, k, v = make_qkv(wl, device="cuda")
+    sc = lbsa.lbsa_score(q, k, wl.block)
+    bs = lbsa.lbsa_select(sc, wl.block, P, "row")
+    emit(workload="tiny", stage="score_f32", **_timer(lambda: lbsa.lbsa_score(q, k, wl.block, scores=sc)))
+    emit(workload="tiny", stage="select_row", **_timer(lambda: lbsa.lbsa_select(sc, wl.block, P, "row")))
+    emit(workload="tiny", stage="attend_f32", **_timer(lambda: lbsa.lbsa_attend(q, k, v, bs)))
+
+    # Wan-like layer, exact mass, 3D tiles
+    wl = get_workload("wan")
+    T, H, W = wl.grid
+    q, k, v = make_qkv(wl, device="cuda")
+    perm = lbsa.lbsa_partition_perm(T, H, W, "3d", device="cuda")
+    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+    sc = lbsa.lbsa_score(qp, kp, wl.block)
+    bs = lbsa.lbsa_select(sc, wl.block, P, "row")
+    fl, _ = flops_of(bs, wl)
+    qkv_bytes = 3 * q.numel() * q.element_size()
+    t = _timer(lambda: lbsa.lbsa_permute([q, k, v], perm, outs=[qp, kp, vp]), flush=flush)
+    emit(workload="wan", stage="permute_qkv", **t, **hbm(2 * qkv_bytes, t["median"]))
+    t = _timer(lambda: lbsa.lbsa_score(qp, kp, wl.block, scores=sc))
+    emit(workload="wan", stage="score_exact", **t, **tfl(2.0 * wl.n_valid ** 2 * wl.d * wl.H, t["median"]))
+    t = _timer(lambda: lbsa.lbsa_select(sc, wl.block, P, "row"), flush=flush)
+    emit(workload="wan", stage="select_row", **t, **hbm(sc.numel() * 4, t["median"]))
+    t = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+    emit(workload="wan", stage="attend", density=fl / (4.0 * wl.d * wl.n_valid ** 2 * wl.H), **t, **tfl(fl, t["median"]))
+    dense = lbsa.lbsa_select(sc, wl.block, 1.0, "row")
+    fld, _ = flops_of(dense, wl)
+    t = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, dense))
+    emit(workload="wan", stage="attend_dense_p1", **t, **tfl(fld, t["median"]))
+    t = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp))
+    emit(workload="wan", stage="torch_sdpa_dense (library reference)", **t, **tfl(fld, t["median"]))
+    del q, k, v, qp, kp, vp, sc, bs, dense
+
+    # skewed heads: p sweep
+    wl = get_workload("wan_skew")
+    q, k, v = make_qkv(wl, device="cuda")
+    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+    sc = lbsa.lbsa_score(qp, kp, wl.block)
+    for p in wl.extra["p_sweep"]:
+        bs = lbsa.lbsa_select(sc, wl.block, p, "row")
+        fl, m = flops_of(bs, wl)
+        ta = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+        ts = _timer(lambda: lbsa.lbsa_select(sc, wl.block, p, "row"), flush=flush)
+        emit(workload="wan_skew", stage="attend", p=p, density=float(m.mean()),
+             density_per_head=[round(float(x), 4) for x in m.mean(axis=(1, 2))], **ta, **tfl(fl, ta["median"]),
+             select_ms=ts["median"])
+    del q, k, v, qp, kp, vp, sc
+
+    # proxy mode: 1D / 2D / 3D cycle, head-scope selection at tau = 0.25
+    wl = get_workload("wan_proxy")
+    q, k, v = make_qkv(wl, device="cuda")
+    for call in range(3):
+        kind = ("1d", "2d", "3d")[call]
+        perm = lbsa.lbsa_partition_perm(T, H, W, kind, device="cuda")
+        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+        sc = lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool")
+        bs = lbsa.lbsa_select(sc, wl.block, 0.25, "head")
+        fl, m = flops_of(bs, wl)
+
+        def full_call():
+            a, b_, c = lbsa.lbsa_permute([q, k, v], perm)
+            s2 = lbsa.lbsa_score(a, b_, wl.block, mode="meanpool")
+            bsx = lbsa.lbsa_select(s2, wl.block, 0.25, "head")
+            o = lbsa.lbsa_attend(a, b_, c, bsx)
+            lbsa.lbsa_permute([o], perm, inverse=True)
+
+        tm = _timer(lambda: lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool", scores=sc), flush=flush)
+        th = _timer(lambda: lbsa.lbsa_select(sc, wl.block, 0.25, "head"), flush=flush)
+        ta = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+        tc = _timer(full_call, flush=flush)
+        empty = float((m.sum(axis=2) == 0).mean())
+        emit(workload="wan_proxy", partition=kind, stage="meanpool", **tm, **hbm(2 * q.numel() * 2 + sc.numel() * 4, tm["median"]))
+        emit(workload="wan_proxy", partition=kind, stage="select_head", **th, **hbm(3 * sc.numel() * 4, th["median"]))
+        emit(workload="wan_proxy", partition=kind, stage="attend", density=float(m.mean()), empty_rows=empty, **ta,
+             **tfl(fl, ta["median"]))
+        emit(workload="wan_proxy", partition=kind, stage="full_call", **tc)
+    del q, k, v, qp, kp, vp, sc
+
+    # HunyuanVideo-like layer: select once, 49 re-drawn attend calls on the frozen blockset
+    wl = get_workload("hunyuan")
+    q32, k32, v32 = make_qkv_f32(wl, device="cuda")
+    q, k, v = (x.to(torch.bfloat16) for x in (q32, k32, v32))
+    t = _timer(lambda: lbsa.lbsa_score(q, k, wl.block), n=3, warm=1)
+    sc = lbsa.lbsa_score(q, k, wl.block)
+    emit(workload="hunyuan", stage="score_exact", **t, **tfl(2.0 * wl.n_valid ** 2 * wl.d * wl.H, t["median"]))
+    bs = lbsa.lbsa_select(sc, wl.block, P, "row")
+    t = _timer(lambda: lbsa.lbsa_select(sc, wl.block, P, "row"), flush=flush)
+    emit(workload="hunyuan", stage="select_row", **t, **hbm(sc.numel() * 4, t["median"]))
+    fl, m = flops_of(bs, wl)
+    times = []
+    for step in range(1, wl.extra["steps"] + 1):
+        q, k, v = redraw_qkv(wl, q32, k32, v32, step)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lbsa.lbsa_attend(q, k, v, bs)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ts = sorted(times)
+    med = ts[len(ts) // 2]
+    emit(workload="hunyuan", stage="attend_frozen_x49", density=float(m.mean()), median=med, p10=ts[4], p90=ts[44],
+         **tfl(fl, med))
+    dense = lbsa.lbsa_select(sc, wl.block, 1.0, "row")
+    fld, _ = flops_of(dense, wl)
+    t = _timer(lambda: lbsa.lbsa_attend(q, k, v, dense), n=3, warm=1)
+    emit(workload="hunyuan", stage="attend_dense_p1", **t, **tfl(fld, t["median"]))
+    t = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(q, k, v), n=3, warm=1)
+    emit(workload="hunyuan", stage="torch_sdpa_dense (library reference)", **t, **tfl(fld, t["median"]))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -369,9 +562,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=["attend", "score", "select"],
                     help="run the small ncu case for one kernel instead of the benchmark")
+    ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
     args = ap.parse_args()
     if args.profile:
         return run_profile(args.profile)
+    if args.sweep:
+        return run_sweep(args)
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
