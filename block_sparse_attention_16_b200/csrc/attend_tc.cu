@@ -18,8 +18,8 @@
 //              per column) back over the first 32 columns of the same S
 //              buffer, rescales O in TMEM when the running max grows by more
 //              than 2^8, and writes the output.
-//   warp 4     TMA producer: Q once, then K and V 64-key tiles through a
-//              2-stage ring.
+//   warp 4     TMA producer: Q once, then K and V 64-key tiles through two
+//              separate 2-stage rings, each refilled as soon as its slot frees.
 //   warp 5     UMMA issuer: S = Q K^T (M=128, N=64, K=d, both operands in
 //              smem) into one of two TMEM S buffers, then O += P V (M=128,
 //              N=d, K=64, P read from TMEM) into TMEM.
@@ -199,28 +199,47 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         mbar_arrive_expect_tx(bars.q_full, L::Q_BYTES);
         for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, bars.q_full, c * 64, tile * BM, h, bb);
       }
-      int issued = 0;
-      for (int s = 0; s < n_steps; ++s) {
-        const int st = s % NS;
-        const uint32_t ph = (s / NS) & 1;
-        const uint32_t e = sched[s / spb];
-        const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
-        if (s >= NS && !mbar_wait(bars.k_empty + st, ph ^ 1, wl, args.status, abort_flag)) break;
-        uint8_t* sK = smem + L::OFF_K + st * L::KV_BYTES;
-        mbar_arrive_expect_tx(bars.k_full + st, L::KV_BYTES);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, bars.k_full + st, c * 64, key0, h, bb);
-        if (s >= NS && !mbar_wait(bars.v_empty + st, ph ^ 1, wl, args.status, abort_flag)) { issued = s + 1; break; }
-        uint8_t* sV = smem + L::OFF_V + st * L::KV_BYTES;
-        mbar_arrive_expect_tx(bars.v_full + st, L::KV_BYTES);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(sV + c * BK * 128, &tmap_v, bars.v_full + st, c * 64, key0, h, bb);
-        issued = s + 1;
+      // K and V stream through separate rings: K stage s is free once S = Q K^T
+      // of step s - NS has completed, V stage s once O += P V of step s - NS
+      // has.  Both slots are probed without blocking so that a K load never
+      // queues behind a V stage that the softmax still holds.
+      int sk = 0, sv = 0;
+      uint64_t t_last = globaltimer_ns();
+      while (sv < n_steps) {
+        const bool k_free = sk < n_steps && (sk < NS || mbar_test_wait(bars.k_empty + sk % NS, ((sk / NS) & 1) ^ 1));
+        const bool v_free = sv < sk && (sv < NS || mbar_test_wait(bars.v_empty + sv % NS, ((sv / NS) & 1) ^ 1));
+        // K of step s+1 is consumed before V of step s: prefer it while it is at most one step ahead
+        const bool do_k = k_free && (sk <= sv + 1 || !v_free);
+        if (do_k || v_free) {
+          const int s = do_k ? sk : sv;
+          const int st = s % NS;
+          const uint32_t e = sched[s / spb];
+          const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
+          if (do_k) {
+            uint8_t* sK = smem + L::OFF_K + st * L::KV_BYTES;
+            mbar_arrive_expect_tx(bars.k_full + st, L::KV_BYTES);
+            for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, bars.k_full + st, c * 64, key0, h, bb);
+            ++sk;
+          } else {
+            uint8_t* sV = smem + L::OFF_V + st * L::KV_BYTES;
+            mbar_arrive_expect_tx(bars.v_full + st, L::KV_BYTES);
+            for (int c = 0; c < D / 64; ++c) tma_load_4d(sV + c * BK * 128, &tmap_v, bars.v_full + st, c * 64, key0, h, bb);
+            ++sv;
+          }
+          t_last = globaltimer_ns();
+          continue;
+        }
+        if (*abort_flag) break;
+        if (globaltimer_ns() - t_last > static_cast<uint64_t>(wl)) {
+          raise_status(args.status, LBSA_ERR_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
       }
       if (*abort_flag) {
         // let copies still in flight land before the CTA can exit
-        for (int s = (issued > NS ? issued - NS : 0); s < issued; ++s) {
-          mbar_wait(bars.k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
-          mbar_wait(bars.v_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
-        }
+        for (int s = (sk > NS ? sk - NS : 0); s < sk; ++s) mbar_wait(bars.k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
+        for (int s = (sv > NS ? sv - NS : 0); s < sv; ++s) mbar_wait(bars.v_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
       }
     }
   } else if (warp == 5) {
