@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
-    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait",
+    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2",
     "lbsa_select_head_noalloc", "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
@@ -84,6 +84,7 @@ def load_library():
         "lbsa_permute": (ctypes.c_int, [ctypes.POINTER(P), ctypes.POINTER(P), I32, P,
                                         ctypes.POINTER(_Desc), I32, P]),
         "lbsa_selftest_wait": (ctypes.c_int, [I64, P, P]),
+        "lbsa_selftest_exp2": (ctypes.c_int, [P, P, I64, P]),
         "lbsa_select_head_noalloc": (ctypes.c_int, [P, I32, I32, I32, D, P, P, P, P]),
         "lbsa_last_error": (ctypes.c_char_p, []),
         "lbsa_version": (ctypes.c_int, []),
@@ -285,6 +286,16 @@ def lbsa_selftest_wait(limit_us: int = 1000, stream=None) -> int:
     out = torch.zeros(1, dtype=torch.int32, device="cuda")
     _check(load_library().lbsa_selftest_wait(limit_us, _ptr(out), _stream(stream)))
     return int(out.item())
+
+
+def lbsa_selftest_exp2(v, stream=None):
+    """2^v through the scorer's FMA-pipe exponential (float32 CUDA tensor)."""
+    if v.dtype != torch.float32 or not v.is_cuda:
+        raise TypeError("v must be a float32 CUDA tensor")
+    v = v.contiguous()
+    out = torch.empty_like(v)
+    _check(load_library().lbsa_selftest_exp2(_ptr(v), _ptr(out), v.numel(), _stream(stream)))
+    return out
 
 
 def lbsa_select_head_noalloc(scores, p: float, counts=None, cols=None, status=None, stream=None):

@@ -212,7 +212,7 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
     if (desc->dtype == LBSA_BF16) {
       CUtensorMap tq, tk;
       if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
-      if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
+      if ((rc = make_tmap(&tk, k, desc, 128)) != LBSA_OK) return rc;
       if ((rc = scratch_alloc(ds, lbsa::score_exact_bf16_workspace_bytes(desc->B, desc->H, desc->N_valid), s, &ws)) !=
           LBSA_OK)
         return rc;
@@ -421,6 +421,15 @@ int lbsa_selftest_wait(int64_t limit_us, int32_t* device_out, void* stream) {
   return LBSA_OK;
 }
 
+int lbsa_selftest_exp2(const float* v, float* out, int64_t n, void* stream) {
+  if (n < 0) return fail(LBSA_ERR_INVALID_ARG, "n < 0");
+  if (n == 0) return LBSA_OK;
+  if (!v || !out) return fail(LBSA_ERR_INVALID_ARG, "v or out is NULL");
+  cudaError_t e = lbsa::launch_selftest_exp2(v, out, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_selftest_exp2 launch");
+  return LBSA_OK;
+}
+
 }  // extern "C"
 
 namespace lbsa {
@@ -448,6 +457,27 @@ __global__ void selftest_wait_kernel(long long limit_ns, int32_t* out) {
 
 cudaError_t launch_selftest_wait(long long limit_ns, int32_t* out, cudaStream_t s) {
   selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, out);
+  return cudaGetLastError();
+}
+
+namespace {
+// pairs through exp2_poly2; an odd tail element is paired with itself
+__global__ void selftest_exp2_kernel(const float* __restrict__ v, float* __restrict__ out, long long n) {
+  for (long long i = 2 * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+       i += 2ll * gridDim.x * blockDim.x) {
+    const float a = v[i], b = (i + 1 < n) ? v[i + 1] : a;
+    float ra, rb;
+    u64_as_f2(exp2_poly2(f2_as_u64(a, b)), ra, rb);
+    out[i] = ra;
+    if (i + 1 < n) out[i + 1] = rb;
+  }
+}
+}  // namespace
+
+cudaError_t launch_selftest_exp2(const float* v, float* out, long long n, cudaStream_t s) {
+  const long long pairs = (n + 1) / 2;
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>((pairs + 255) / 256, 4096));
+  selftest_exp2_kernel<<<blocks, 256, 0, s>>>(v, out, n);
   return cudaGetLastError();
 }
 }  // namespace lbsa

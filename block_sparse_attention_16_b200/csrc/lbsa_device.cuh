@@ -255,6 +255,31 @@ __device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsign
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+
+// 2^v for a pair of v <= 0 on the FMA pipe (no MUFU): v = j + f with
+// j = rint(v) (round-to-nearest by adding 1.5 * 2^23, whose ulp is 1) and
+// f in [-1/2, 1/2]; 2^f from a degree-4 polynomial fitted to minimise the
+// relative error on [-1/2, 1/2] (iteratively reweighted least squares on
+// Chebyshev nodes: 2.6e-6 in exact arithmetic, 2.7e-6 evaluated in fp32);
+// 2^j is added to the exponent field.  Inputs below -125 are clamped there
+// (the result, < 2^-124, only ever adds to a sum that holds a term >= 1).
+__device__ __forceinline__ unsigned long long exp2_poly2(unsigned long long v2) {
+  float a, b;
+  u64_as_f2(v2, a, b);
+  const unsigned long long v = f2_as_u64(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const unsigned long long t = fadd2(v, f2_as_u64(12582912.f, 12582912.f));     // low bits: rint(v)
+  const unsigned long long jf = fadd2(t, f2_as_u64(-12582912.f, -12582912.f));
+  const unsigned long long f = ffma2(jf, f2_as_u64(-1.f, -1.f), v);
+  unsigned long long q = ffma2(f2_as_u64(0.009570096619427204f, 0.009570096619427204f), f,
+                               f2_as_u64(0.05591785907745361f, 0.05591785907745361f));
+  q = ffma2(q, f, f2_as_u64(0.240247443318367f, 0.240247443318367f));
+  q = ffma2(q, f, f2_as_u64(0.6931217908859253f, 0.6931217908859253f));
+  q = ffma2(q, f, f2_as_u64(0.9999992847442627f, 0.9999992847442627f));
+  // bits(t) << 23 == j << 23 (mod 2^32): the constant's bits vanish in the shift
+  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
+  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+  return (static_cast<unsigned long long>(hi) << 32) | lo;
+}
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

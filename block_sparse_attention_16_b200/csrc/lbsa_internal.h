@@ -81,6 +81,7 @@ cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, co
                            const lbsa_qkv_desc& d, int inverse, cudaStream_t s);
 
 cudaError_t launch_selftest_wait(long long limit_ns, int32_t* out, cudaStream_t s);
+cudaError_t launch_selftest_exp2(const float* v, float* out, long long n, cudaStream_t s);
 
 // Records `msg` as this thread's lbsa_last_error() text and returns `code`.
 int set_error(int code, const char* msg);

@@ -15,23 +15,31 @@
 // and every exponential of the dense pass is computed once.
 //
 // Persistent grid (two CTAs per SM, each walking tiles with a grid stride), so
-// the scratch is bounded: gridDim.x * 128 * n_chunks floats.  Each thread
-// reads back only the scratch values it wrote itself.
+// the scratch is bounded: gridDim.x * (128 + 4) * n_chunks floats.  Each
+// thread reads back only the strip values it wrote itself.
 //
 // Warp roles (192 threads): warps 0-3 softmax (thread t = tile row t = TMEM
-// lane t), warp 4 TMA producer (Q per tile, K 64-key tiles through a ring),
-// warp 5 UMMA issuer (S = Q K^T, M=128, N=64, K=d, double-buffered in TMEM
-// columns [0,64) and [64,128)).
+// lane t), warp 4 TMA producer (Q per tile, K 128-key tiles through a ring),
+// warp 5 UMMA issuer (S = Q K^T, M=128, N=128, K=d, double-buffered in TMEM
+// columns [0,128) and [128,256)).  One step covers two 64-key chunks; the
+// 128-wide UMMA keeps the tensor pipe's per-instruction cost amortised.
 #include "lbsa_device.cuh"
 
 namespace lbsa {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;
-constexpr int NS = 3;
+constexpr int BK = 128;           // keys per UMMA step
+constexpr int CH = 64;            // keys per chunk (one mass entry per 64-key chunk)
+constexpr int NS = 2;
+// Of every 8 exponential pairs of a full chunk, those whose bit is set take
+// the FMA-pipe exponential (exp2_poly2) instead of MUFU ex2: a quarter of the
+// exponentials moves off the MUFU, which otherwise bounds the softmax warps.
+#ifndef LBSA_SCORE_POLY_MASK
+#define LBSA_SCORE_POLY_MASK 0x88
+#endif
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 256;
 constexpr int kCtasPerSm = 2;
 template <int D>
 struct Layout {
@@ -43,8 +51,7 @@ struct Layout {
   // q_full, q_empty, k_full[NS], k_empty[NS], s_full[2], s_free[2], drain
   static constexpr int NBAR = 2 + 2 * NS + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_PART = OFF_MISC + 16;
-  static size_t bytes(int n_chunks) { return OFF_PART + static_cast<size_t>(4) * n_chunks * 4 + 1024; }
+  static size_t bytes() { return OFF_MISC + 16 + 1024; }
 };
 
 struct TileIdx {
@@ -68,7 +75,8 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int N = args.N_valid;
-  const int n_chunks = (N + BK - 1) / BK;
+  const int n_chunks = (N + CH - 1) / CH;
+  const int n_steps = (N + BK - 1) / BK;
   const int tiles_per_bh = (N + BM - 1) / BM;
   const int total_tiles = tiles_per_bh * args.H * args.B;
   const long long wl = args.wait_limit;
@@ -84,7 +92,9 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
   uint64_t* drain = s_free + 2;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  float* part = reinterpret_cast<float*>(smem + L::OFF_PART);   // [4][n_chunks]
+  // per-warp chunk partials of the current tile: [4][n_chunks] after the strips
+  float* part = args.scratch + static_cast<long long>(gridDim.x) * n_chunks * BM +
+                static_cast<long long>(blockIdx.x) * 4 * n_chunks;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -124,7 +134,7 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
         if (it >= 1 && !mbar_wait(q_empty, (it - 1) & 1, wl, args.status, abort_flag)) break;
         mbar_arrive_expect_tx(q_full, L::Q_BYTES);
         for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, q_full, c * 64, t.tile * BM, t.h, t.bb);
-        for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+        for (int j = 0; j < n_steps; ++j, ++s) {
           const int st = static_cast<int>(s % NS);
           if (s >= NS && !mbar_wait(k_empty + st, static_cast<uint32_t>((s / NS) & 1) ^ 1u, wl, args.status, abort_flag)) {
             ok = false;
@@ -132,7 +142,7 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
           }
           uint8_t* sK = smem + L::OFF_K + st * L::K_BYTES;
           mbar_arrive_expect_tx(k_full + st, L::K_BYTES);
-          for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, ch * BK, t.h, t.bb);
+          for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, j * BK, t.h, t.bb);
         }
       }
       if (*abort_flag) {
@@ -152,7 +162,7 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
       bool ok = true;
       for (int g = blockIdx.x; ok && g < total_tiles; g += gridDim.x, ++it) {
         if (!mbar_wait(q_full, it & 1, wl, args.status, abort_flag)) break;
-        for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+        for (int j = 0; j < n_steps; ++j, ++s) {
           const int st = static_cast<int>(s % NS);
           const int sb = static_cast<int>(s & 1);
           if (!mbar_wait(k_full + st, static_cast<uint32_t>((s / NS) & 1), wl, args.status, abort_flag) ||
@@ -189,58 +199,71 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
       const int grow = t.tile * BM + row;
       const bool valid_row = grow < N;
       float m = -INFINITY, l = 0.f;
-      for (int ch = 0; ch < n_chunks; ++ch, ++s) {
+      for (int j = 0; j < n_steps && alive; ++j, ++s) {
         const int sb = static_cast<int>(s & 1);
         if (!mbar_wait(s_full + sb, static_cast<uint32_t>((s >> 1) & 1), wl, args.status, abort_flag)) {
           alive = false;
           break;
         }
         tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(s_free + sb);
-        const int nvk = N - ch * BK;
-        // row max of the raw logits (the scale is positive), 4 independent chains
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (nvk >= 64) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 2)
-            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < nvk) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(r[c]));
-        }
-        const float m_new = fmaxf(m, fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2);
-        // sum of 2^(s*scale - m_new): packed FMA per pair, MUFU ex2, packed adds
-        const unsigned long long sc2 = f2_as_u64(scale_log2, scale_log2);
-        const unsigned long long nm2 = f2_as_u64(-m_new, -m_new);
-        unsigned long long acc4[4] = {0ull, 0ull, 0ull, 0ull};
-        if (nvk >= 64) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v0, v1;
-            u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
-            acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(ex2(v0), ex2(v1)));
+        const int nh = min(2, n_chunks - 2 * j);      // chunks in this step (block-uniform)
+        for (int hf = 0; hf < nh; ++hf) {
+          const int ch = 2 * j + hf;
+          uint32_t r[64];
+          tmem_ld32(t_lane + sb * BK + hf * CH, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(t_lane + sb * BK + hf * CH + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          tmem_wait_ld();
+          if (hf == nh - 1) {
+            // the whole S buffer is in registers: the UMMA may overwrite it
+            tc_fence_before();
+            mbar_arrive(s_free + sb);
           }
-        } else {
+          const int nvk = N - ch * CH;
+          // row max of the raw logits (the scale is positive), 4 independent chains
+          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (nvk >= 64) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float v0, v1;
-            u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
-            acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(2 * c < nvk ? ex2(v0) : 0.f, 2 * c + 1 < nvk ? ex2(v1) : 0.f));
+            for (int c = 0; c < 64; c += 2)
+              mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c < nvk) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(r[c]));
           }
-        }
-        float a8[8];
+          const float m_new = fmaxf(m, fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2);
+          // sum of 2^(s*scale - m_new): packed FMA per pair, MUFU ex2 (or the
+          // FMA-pipe exponential for the pairs LBSA_SCORE_POLY_MASK picks), packed adds
+          const unsigned long long sc2 = f2_as_u64(scale_log2, scale_log2);
+          const unsigned long long nm2 = f2_as_u64(-m_new, -m_new);
+          unsigned long long acc4[4] = {0ull, 0ull, 0ull, 0ull};
+          if (nvk >= 64) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) u64_as_f2(acc4[i], a8[2 * i], a8[2 * i + 1]);
-        const float bsum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-        l = (m == -INFINITY) ? bsum : fmaf(l, ex2(m - m_new), bsum);
-        m = m_new;
-        strip[static_cast<long long>(ch) * BM + row] = m + __log2f(bsum);
+            for (int c = 0; c < 32; ++c) {
+              float v0, v1;
+              const unsigned long long v2 = ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2);
+              if ((LBSA_SCORE_POLY_MASK >> (c & 7)) & 1) {
+                acc4[c & 3] = fadd2(acc4[c & 3], exp2_poly2(v2));
+              } else {
+                u64_as_f2(v2, v0, v1);
+                acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(ex2(v0), ex2(v1)));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              float v0, v1;
+              u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
+              acc4[c & 3] = fadd2(acc4[c & 3], f2_as_u64(2 * c < nvk ? ex2(v0) : 0.f, 2 * c + 1 < nvk ? ex2(v1) : 0.f));
+            }
+          }
+          float a8[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) u64_as_f2(acc4[i], a8[2 * i], a8[2 * i + 1]);
+          const float bsum = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+          l = (m == -INFINITY) ? bsum : fmaf(l, ex2(m - m_new), bsum);
+          m = m_new;
+          strip[static_cast<long long>(ch) * BM + row] = m + __log2f(bsum);
+        }
       }
       if (!alive) break;
       const float lse2 = m + __log2f(l);
@@ -319,24 +342,23 @@ int score_grid(int N, int H, int B) {
 }  // namespace
 
 size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid) {
-  const int n_chunks = (N_valid + BK - 1) / BK;
-  return static_cast<size_t>(score_grid(N_valid, H, B)) * BM * n_chunks * sizeof(float) + 256;
+  const int n_chunks = (N_valid + CH - 1) / CH;
+  return static_cast<size_t>(score_grid(N_valid, H, B)) * (BM + 4) * n_chunks * sizeof(float) + 256;
 }
 
 cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
                                     cudaStream_t s) {
-  const int n_chunks = (a.N_valid + BK - 1) / BK;
   dim3 grid(score_grid(a.N_valid, a.H, a.B));
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
   if (a.d == 128) {
-    const size_t smem = Layout<128>::bytes(n_chunks);
+    const size_t smem = Layout<128>::bytes();
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_exact_bf16_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     score_exact_bf16_kernel<128><<<grid, kThreads, smem, s>>>(*tq, *tk, a, scale_log2);
   } else {
-    const size_t smem = Layout<64>::bytes(n_chunks);
+    const size_t smem = Layout<64>::bytes();
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(score_exact_bf16_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

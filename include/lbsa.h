@@ -201,6 +201,14 @@ int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const in
  * and writes LBSA_ERR_TIMEOUT to *device_out (device int32).  Never hangs. */
 int lbsa_selftest_wait(int64_t limit_us, int32_t* device_out, void* stream);
 
+/* Self-test of the FMA-pipe exponential the exact scorer uses for a quarter
+ * of its exponentials: out[i] = 2^v[i] for n device floats v[i] <= 0, by
+ * round-to-nearest range reduction and a degree-4 polynomial on [-1/2, 1/2]
+ * (relative error below 3e-6 for v in [-125, 0]; inputs below -125 give
+ * 2^-125).  v and out are device float arrays of n elements (n >= 0); they
+ * may alias.  Returns LBSA_ERR_INVALID_ARG on a NULL pointer with n > 0. */
+int lbsa_selftest_exp2(const float* v, float* out, int64_t n, void* stream);
+
 /* Head-scope selection that allocates nothing (the pages have no
  * counterpart).  It serves callers that cannot call cudaMalloc: a host
  * framework whose own caching allocator owns the device's memory (a

@@ -253,3 +253,18 @@ def test_meanpool_head_scope_pipeline(dtype):
     assert_csr_equal(csr, oracle.select_contract(host(scores), 0.25, "head"))
     ref_o, _ = oracle.sparse_attention(qh, kh, vh, wl.n_valid, wl.block, *csr)
     assert_out_close(host(out), ref_o[:, :, :wl.n_valid], q.dtype)
+
+
+@pytest.mark.gpu
+def test_fma_pipe_exp2_within_its_error_bound():
+    """The scorer's FMA-pipe exponential against 2^v in fp64 over its domain."""
+    v = torch.cat([torch.linspace(-125.0, 0.0, 1_000_001, dtype=torch.float64),
+                   -30.0 * torch.rand(200_001, dtype=torch.float64, generator=torch.Generator().manual_seed(7)),
+                   torch.tensor([-0.5, 0.5 - 1.0, -1e-30, 0.0], dtype=torch.float64)]).float()
+    out = lbsa.lbsa_selftest_exp2(v.cuda()).cpu().double()
+    ref = torch.exp2(v.double())
+    rel = ((out - ref).abs() / ref).max().item()
+    assert rel < 3e-6, rel
+    # below the clamp the result is 2^-125 (tiny, never negative or garbage)
+    low = lbsa.lbsa_selftest_exp2(torch.tensor([-126.0, -500.0, -1e30], device="cuda")).cpu().double()
+    assert torch.all((low - 2.0 ** -125).abs() <= 1e-6 * 2.0 ** -125), low
