@@ -79,10 +79,15 @@ class Clocks:
         try:
             self.f = open(path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # start timing only once the sampler is writing (nvidia-smi takes a moment to start)
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(path) == 0 and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -362,7 +367,8 @@ def load_traffic(kernel):
 
 def run_profile(kernel):
     """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
-    than L2), one warm-up pass of the path, then two launches of `kernel`."""
+    than L2), one warm-up pass of the path, then two launches of `kernel`; or,
+    for "proxy", one mean-pooled proxy call per partition on the full shape."""
     import dataclasses
 
     import block_sparse_attention_16_b200 as lbsa
@@ -370,6 +376,21 @@ def run_profile(kernel):
     from block_sparse_attention_16_b200.workload import get_workload, make_qkv
 
     build()
+    if kernel == "proxy":
+        # mean-pooled proxy path of the Wan-like shape, one call per partition
+        wl = get_workload("wan_proxy")
+        T, H, W = wl.grid
+        q, k, v = make_qkv(wl, device="cuda")
+        for part in ("1d", "2d", "3d"):
+            perm = lbsa.lbsa_partition_perm(T, H, W, part, device="cuda")
+            qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+            sc = lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool")
+            bs = lbsa.lbsa_select(sc, wl.block, wl.p, "head")
+            lbsa.lbsa_attend(qp, kp, vp, bs)
+        torch.cuda.synchronize()
+        assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+        print("profile case proxy: ok")
+        return 0
     wl = dataclasses.replace(get_workload(WORKLOAD), H=6)
     T, H, W = wl.grid
     q, k, v = make_qkv(wl, device="cuda")
@@ -556,11 +577,11 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["attend", "score", "select"],
+    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy"],
                     help="run the small ncu case for one kernel instead of the benchmark")
     ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
     args = ap.parse_args()
