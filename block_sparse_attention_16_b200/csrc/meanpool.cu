@@ -46,14 +46,21 @@ __global__ void block_mean_kernel(const T* __restrict__ q, const T* __restrict__
   const int r0 = i * block, r1 = min(r0 + block, desc.N_valid);
   const long long base = bb * desc.stride_b + h * desc.stride_h;
   float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int r = r0 + g; r < r1; r += G) {
-    float f[8];
-    load8(q + base + r * desc.stride_n + v * 8, f);
+  // at most 128 / G rows per thread: unrolled and predicated, so that all of a
+  // thread's 16-byte loads are in flight together
+  constexpr int kMaxIt = 128 / G;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) aq[e] += f[e];
-    load8(k + base + r * desc.stride_n + v * 8, f);
+  for (int it = 0; it < kMaxIt; ++it) {
+    const int r = r0 + g + it * G;
+    if (r < r1) {
+      float f[8];
+      load8(q + base + r * desc.stride_n + v * 8, f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ak[e] += f[e];
+      for (int e = 0; e < 8; ++e) aq[e] += f[e];
+      load8(k + base + r * desc.stride_n + v * 8, f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ak[e] += f[e];
+    }
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
@@ -72,38 +79,48 @@ __global__ void block_mean_kernel(const T* __restrict__ q, const T* __restrict__
 }
 
 // grid (nT, nT, B*H) with nT = ceil(nB/64); 256 threads, each a 4x4 patch of s.
+// Column chunks of qbar and kbar are staged transposed ([c][row]) so that a
+// thread reads its 4 rows and its 4 columns as one 16-byte load each.
 template <int D>
-__global__ void logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar, int nB, float scale,
-                              float* __restrict__ scores, float2* __restrict__ part) {
+__global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ qbar, const float* __restrict__ kbar,
+                                                     int nB, float scale, float* __restrict__ scores,
+                                                     float2* __restrict__ part) {
   constexpr int KC = 32;                 // columns of d staged per round
-  __shared__ float sq[kTile][KC + 1];
-  __shared__ float sk[kTile][KC + 1];
-  __shared__ float red_m[256], red_s[256];
+  constexpr int LD = kTile + 4;          // row stride of the staged chunks (16-byte aligned rows)
+  __shared__ __align__(16) float sq[KC][LD];
+  __shared__ __align__(16) float sk[KC][LD];
+  __shared__ float red_m[8], red_s[8];
   const int ti = blockIdx.y, tj = blockIdx.x, g = blockIdx.z;
   const int nT = gridDim.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* qb = qbar + static_cast<long long>(g) * nB * D;
   const float* kb = kbar + static_cast<long long>(g) * nB * D;
   const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
   float acc[4][4] = {};
   for (int c0 = 0; c0 < D; c0 += KC) {
-    for (int e = threadIdx.x; e < kTile * KC; e += 256) {
-      const int r = e / KC, c = e % KC;
+    // 64 rows x 8 float4 per operand: two float4 per thread per operand
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int e = threadIdx.x + it * 256;
+      const int r = e >> 3, c4 = (e & 7) * 4;
       const int qi = ti * kTile + r, kj = tj * kTile + r;
-      sq[r][c] = (qi < nB) ? qb[static_cast<long long>(qi) * D + c0 + c] : 0.f;
-      sk[r][c] = (kj < nB) ? kb[static_cast<long long>(kj) * D + c0 + c] : 0.f;
+      const float4 a = (qi < nB) ? *reinterpret_cast<const float4*>(qb + static_cast<long long>(qi) * D + c0 + c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 b = (kj < nB) ? *reinterpret_cast<const float4*>(kb + static_cast<long long>(kj) * D + c0 + c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      sq[c4][r] = a.x; sq[c4 + 1][r] = a.y; sq[c4 + 2][r] = a.z; sq[c4 + 3][r] = a.w;
+      sk[c4][r] = b.x; sk[c4 + 1][r] = b.y; sk[c4 + 2][r] = b.z; sk[c4 + 3][r] = b.w;
     }
     __syncthreads();
+#pragma unroll 8
     for (int c = 0; c < KC; ++c) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[u] = sq[tr + u][c];
-        b[u] = sk[tc + u][c];
-      }
+      const float4 a = *reinterpret_cast<const float4*>(&sq[c][tr]);
+      const float4 b = *reinterpret_cast<const float4*>(&sk[c][tc]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(a[u], b[w], acc[u][w]);
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
     }
     __syncthreads();
   }
@@ -119,13 +136,13 @@ __global__ void logits_kernel(const float* __restrict__ qbar, const float* __res
         mx = fmaxf(mx, acc[u][w]);
       }
     }
-  red_m[threadIdx.x] = mx;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red_m[warp] = mx;
   __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red_m[threadIdx.x] = fmaxf(red_m[threadIdx.x], red_m[threadIdx.x + o]);
-    __syncthreads();
-  }
-  const float tm = red_m[0];
+  float tm = red_m[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) tm = fmaxf(tm, red_m[w]);
   float sm = 0.f;
 #pragma unroll
   for (int u = 0; u < 4; ++u)
@@ -134,28 +151,38 @@ __global__ void logits_kernel(const float* __restrict__ qbar, const float* __res
       const int qi = ti * kTile + tr + u, kj = tj * kTile + tc + w;
       if (qi < nB && kj < nB) sm += expf(acc[u][w] - tm);
     }
-  red_s[threadIdx.x] = sm;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+  if (lane == 0) red_s[warp] = sm;
   __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red_s[threadIdx.x] += red_s[threadIdx.x + o];
-    __syncthreads();
+  if (threadIdx.x == 0) {
+    float z = 0.f;
+    for (int w = 0; w < 8; ++w) z += red_s[w];
+    part[(static_cast<long long>(g) * nT + ti) * nT + tj] = make_float2(tm, z);
   }
-  if (threadIdx.x == 0) part[(static_cast<long long>(g) * nT + ti) * nT + tj] = make_float2(tm, red_s[0]);
 }
 
-// grid (chunks, B*H), 256 threads: combine the head's tile partials (fixed
-// order), then normalise a chunk of the head's scores in place.
+// grid (chunks, B*H), 256 threads: warp 0 combines the head's tile partials
+// (fixed order per lane, then a fixed shuffle tree), then the block
+// normalises a chunk of the head's scores in place.
 __global__ void normalize_kernel(float* __restrict__ scores, const float2* __restrict__ part, int nB, int nT) {
   __shared__ float sM, sZ;
   const int g = blockIdx.y;
   const float2* pp = part + static_cast<long long>(g) * nT * nT;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
     float M = -INFINITY;
-    for (int t = 0; t < nT * nT; ++t) M = fmaxf(M, pp[t].x);
+    for (int t = lane; t < nT * nT; t += 32) M = fmaxf(M, pp[t].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Z = 0.f;
-    for (int t = 0; t < nT * nT; ++t) Z += pp[t].y * expf(pp[t].x - M);
-    sM = M;
-    sZ = Z;
+    for (int t = lane; t < nT * nT; t += 32) Z += pp[t].y * expf(pp[t].x - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+    if (lane == 0) {
+      sM = M;
+      sZ = Z;
+    }
   }
   __syncthreads();
   const float M = sM, invZ = 1.0f / sZ;
