@@ -54,24 +54,28 @@ struct PtrPack {
   uint4* y[3];
 };
 
-__global__ void permute_kernel_packed(PtrPack pk, int count, const int32_t* __restrict__ perm, int B, int H, int N,
-                                      int vec_per_row, long long sb, long long sh, long long sn, int inverse) {
-  const long long per_t = static_cast<long long>(B) * H * N * vec_per_row;
-  const long long total = per_t * count;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / per_t);
-    long long r = i - t * per_t;
-    const int v = static_cast<int>(r % vec_per_row);
-    r /= vec_per_row;
-    const int slot = static_cast<int>(r % N);
-    r /= N;
-    const int h = static_cast<int>(r % H);
-    const int b = static_cast<int>(r / H);
+// grid (ceil(N / kPermRows), count * B * H), 256 threads: thread (row r of the
+// CTA's iteration, 16-byte vector v) copies row slots r0 + r, r0 + r + rpi, ...
+// (32-bit row indices; every thread keeps several independent loads in flight).
+constexpr int kPermRows = 64;
+__global__ void __launch_bounds__(256) permute_kernel_packed(PtrPack pk, const int32_t* __restrict__ perm, int B,
+                                                             int H, int N, int vec_per_row, long long sb,
+                                                             long long sh, long long sn, int inverse) {
+  const int tbh = blockIdx.y;                       // tensor * (B*H) + b*H + h
+  const int t = tbh / (B * H);
+  const int bh = tbh - t * (B * H);
+  const int b = bh / H, h = bh - b * H;
+  const long long base = b * sb + h * sh;
+  const uint4* __restrict__ x = pk.x[t];
+  uint4* __restrict__ y = pk.y[t];
+  const int rpi = blockDim.x / vec_per_row;         // rows per iteration
+  const int lr = threadIdx.x / vec_per_row;
+  const int v = threadIdx.x - lr * vec_per_row;
+  const int r0 = blockIdx.x * kPermRows;
+  const int r1 = min(r0 + kPermRows, N);
+#pragma unroll 4
+  for (int slot = r0 + lr; slot < r1; slot += rpi) {
     const int src = __ldg(perm + slot);
-    const long long base = b * sb + h * sh;
-    const uint4* x = pk.x[t];
-    uint4* y = pk.y[t];
     if (!inverse) y[base + slot * sn + v] = __ldg(x + base + src * sn + v);
     else y[base + src * sn + v] = __ldg(x + base + slot * sn + v);
   }
@@ -104,10 +108,13 @@ cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, co
     pk.x[t] = static_cast<const uint4*>(xs[t]);
     pk.y[t] = static_cast<uint4*>(ys[t]);
   }
-  const long long total = static_cast<long long>(count) * d.B * d.H * d.N_valid * vec_per_row;
-  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 148 * 16));
-  permute_kernel_packed<<<blocks, 256, 0, s>>>(pk, count, perm, d.B, d.H, d.N_valid, vec_per_row, d.stride_b / k,
-                                               d.stride_h / k, d.stride_n / k, inverse);
+  // vec_per_row is d * esize / 16 in {8, 16, 32}: it divides the 256 threads
+  if (vec_per_row <= 0 || 256 % vec_per_row != 0) return cudaErrorInvalidValue;
+  const long long ybh = static_cast<long long>(count) * d.B * d.H;
+  if (ybh > 65535) return cudaErrorInvalidValue;
+  dim3 grid((d.N_valid + kPermRows - 1) / kPermRows, static_cast<unsigned>(ybh));
+  permute_kernel_packed<<<grid, 256, 0, s>>>(pk, perm, d.B, d.H, d.N_valid, vec_per_row, d.stride_b / k, d.stride_h / k,
+                                             d.stride_n / k, inverse);
   return cudaGetLastError();
 }
 

@@ -147,18 +147,24 @@ struct HeadState {
 
 constexpr int kDigitBits = 10;
 constexpr int kBins = 1 << kDigitBits;
+constexpr long long kHistPerCta = 4096;     // elements per histogram CTA (256 threads x 16)
 
 // pass 0..2: histogram of weights by digit among elements whose higher digits
 // match the resolved prefix.  grid (chunks, G), 256 threads.
 __global__ void head_hist_kernel(const float* __restrict__ scores, long long seg_len, int pass,
                                  unsigned long long* __restrict__ hist, HeadState* __restrict__ st) {
-  __shared__ unsigned long long sh[kBins];
+  // weights split into 20 low and 13 high bits, summed with 32-bit shared
+  // atomics (a CTA sees at most kHistPerCta elements: the low sums stay < 2^32)
+  __shared__ uint32_t sh_lo[kBins], sh_hi[kBins];
   __shared__ unsigned int smax;
   __shared__ int sbad;
   const int g = blockIdx.y;
   HeadState* s = st + g;
   if (pass > 0 && (s->resolved || s->keep_all)) return;
-  for (int i = threadIdx.x; i < kBins; i += blockDim.x) sh[i] = 0;
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
+    sh_lo[i] = 0u;
+    sh_hi[i] = 0u;
+  }
   if (threadIdx.x == 0) {
     smax = 0;
     sbad = 0;
@@ -179,7 +185,11 @@ __global__ void head_hist_kernel(const float* __restrict__ scores, long long seg
     if (pass == 0) lmax = max(lmax, b);
     if (pass > 0 && (b >> (shift + kDigitBits)) != prefix) continue;
     const uint64_t w = fixed_weight(b);
-    if (w) atomicAdd(&sh[(b >> shift) & (kBins - 1)], static_cast<unsigned long long>(w));
+    if (w) {
+      const uint32_t bin = (b >> shift) & (kBins - 1);
+      atomicAdd(&sh_lo[bin], static_cast<uint32_t>(w & 0xFFFFFull));
+      atomicAdd(&sh_hi[bin], static_cast<uint32_t>(w >> 20));
+    }
   }
   if (pass == 0) {
     atomicMax(&smax, lmax);
@@ -187,8 +197,10 @@ __global__ void head_hist_kernel(const float* __restrict__ scores, long long seg
   }
   __syncthreads();
   unsigned long long* gh = hist + static_cast<long long>(g) * kBins;
-  for (int i = threadIdx.x; i < kBins; i += blockDim.x)
-    if (sh[i]) atomicAdd(gh + i, sh[i]);
+  for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
+    const unsigned long long v = (static_cast<unsigned long long>(sh_hi[i]) << 20) + sh_lo[i];
+    if (v) atomicAdd(gh + i, v);
+  }
   if (threadIdx.x == 0 && pass == 0) {
     atomicMax(&s->maxbits, smax);
     if (sbad) atomicExch(&s->bad, 1);
@@ -447,7 +459,7 @@ cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double
   if (e != cudaSuccess) return e;
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  const int chunks = static_cast<int>(std::min<long long>(64, (seg + 4095) / 4096));
+  const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
   for (int pass = 0; pass < 3; ++pass) {
     head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
     head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, bs->status);
@@ -550,7 +562,7 @@ extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t 
   if (e != cudaSuccess) return set_error(LBSA_ERR_CUDA, cudaGetErrorString(e));
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  const int chunks = static_cast<int>(std::min<long long>(64, (seg + 4095) / 4096));
+  const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
   for (int pass = 0; pass < 3; ++pass) {
     head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
     head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, status);
