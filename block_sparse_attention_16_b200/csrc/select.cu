@@ -142,17 +142,95 @@ struct HeadState {
   int keep_all;
   unsigned int tb;
   unsigned int need;
-  int pad;
+  unsigned int arrived;      // histogram CTAs of the current pass that have finished
 };
 
 constexpr int kDigitBits = 10;
 constexpr int kBins = 1 << kDigitBits;
 constexpr long long kHistPerCta = 4096;     // elements per histogram CTA (256 threads x 16)
 
+// After pass k, run by the last histogram CTA of the head (256 threads, bins
+// 4t .. 4t+3 per thread): pick the digit where the weight at or above crosses
+// T, and clear the histogram for the next pass.
+__device__ void find_digit(int pass, uint32_t Pfix, int keep_all, unsigned long long* __restrict__ gh,
+                           HeadState* __restrict__ s, int32_t* __restrict__ status) {
+  __shared__ unsigned long long warp_tot[8];
+  __shared__ int done;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  unsigned long long v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = __ldcg(gh + 4 * t + i);           // summed by other CTAs' atomics: read from L2
+    gh[4 * t + i] = 0ull;
+  }
+  // suffix sums: thread total, inclusive suffix over the warp's lanes, then over the warps
+  unsigned long long x = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) warp_tot[w] = x;
+  if (t == 0) done = 0;
+  __syncthreads();
+  unsigned long long later = 0;
+  for (int u = w + 1; u < 8; ++u) later += warp_tot[u];
+  unsigned long long S[5];                    // S[i] = weight of bins >= 4t + i
+  S[0] = x + later;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) S[i + 1] = S[i] - v[i];
+  if (t == 0 && pass == 0) {
+    s->W = S[0];
+    if (__ldcg(&s->bad)) {                  // set by other CTAs' atomics this pass
+      raise_status(status, LBSA_ERR_INVALID_SCORES);
+      s->keep_all = 1;
+      done = 1;
+    } else if (keep_all) {
+      s->keep_all = 1;
+      done = 1;
+    } else {
+      s->T = threshold_T(S[0], Pfix);
+      s->above = 0;
+      s->prefix = 0;
+      if (s->T == 0) {
+        s->resolved = 1;
+        s->tb = __ldcg(&s->maxbits);
+        s->need = 1;
+        done = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (done) return;
+  const unsigned long long T = s->T;
+  const unsigned long long above = s->above;
+  const unsigned int prefix = s->prefix;
+  __syncthreads();                            // every thread has read the state before it changes
+  // the largest bin b with above + S(b) >= T (exists: S(0) covers everything not above)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (above + S[i] >= T && above + S[i + 1] < T) {
+      const unsigned int b = static_cast<unsigned int>(4 * t + i);
+      s->above = above + S[i + 1];
+      s->prefix = (prefix << kDigitBits) | b;
+      if (pass == 2) {
+        const unsigned int tb = (prefix << kDigitBits) | b;
+        s->tb = tb;
+        const unsigned long long ww = fixed_weight(tb);
+        s->need = static_cast<unsigned int>((T - (above + S[i + 1]) + ww - 1) / ww);
+        s->resolved = 1;
+      }
+    }
+  }
+}
+
 // pass 0..2: histogram of weights by digit among elements whose higher digits
 // match the resolved prefix.  grid (chunks, G), 256 threads.
-__global__ void head_hist_kernel(const float* __restrict__ scores, long long seg_len, int pass,
-                                 unsigned long long* __restrict__ hist, HeadState* __restrict__ st) {
+__global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict__ scores, long long seg_len, int pass,
+                                                        uint32_t Pfix, int keep_all,
+                                                        unsigned long long* __restrict__ hist,
+                                                        HeadState* __restrict__ st, int32_t* __restrict__ status) {
+  __shared__ int is_last;
   // weights split into 20 low and 13 high bits, summed with 32-bit shared
   // atomics (a CTA sees at most kHistPerCta elements: the low sums stay < 2^32)
   __shared__ uint32_t sh_lo[kBins], sh_hi[kBins];
@@ -205,75 +283,15 @@ __global__ void head_hist_kernel(const float* __restrict__ scores, long long seg
     atomicMax(&s->maxbits, smax);
     if (sbad) atomicExch(&s->bad, 1);
   }
-}
-
-// After pass k: pick the digit where the weight at or above crosses T.
-// grid G, kBins threads.  Clears the histogram for the next pass.
-__global__ void head_find_kernel(int pass, uint32_t Pfix, int keep_all, unsigned long long* __restrict__ hist,
-                                 HeadState* __restrict__ st, int32_t* __restrict__ status) {
-  __shared__ unsigned long long suf[kBins];
-  const int g = blockIdx.x;
-  const int t = threadIdx.x;
-  HeadState* s = st + g;
-  if (pass > 0 && (s->resolved || s->keep_all)) return;
-  unsigned long long* gh = hist + static_cast<long long>(g) * kBins;
-  const unsigned long long v = gh[t];
-  gh[t] = 0;
-  // inclusive suffix sum: suf[t] = sum_{u >= t} v[u]
-  suf[t] = v;
+  // the last CTA of this head to finish resolves the digit (no CTA waits for another)
+  __threadfence();
   __syncthreads();
-  for (int o = 1; o < kBins; o <<= 1) {
-    const unsigned long long add = (t + o < kBins) ? suf[t + o] : 0ull;
-    __syncthreads();
-    suf[t] += add;
-    __syncthreads();
-  }
-  __shared__ int done;
-  if (t == 0) {
-    done = 0;
-    if (pass == 0) {
-      s->W = suf[0];
-      if (s->bad) {
-        raise_status(status, LBSA_ERR_INVALID_SCORES);
-        s->keep_all = 1;
-        done = 1;
-      } else if (keep_all) {
-        s->keep_all = 1;
-        done = 1;
-      } else {
-        const unsigned __int128 num = static_cast<unsigned __int128>(suf[0]) * Pfix + ((1u << 24) - 1);
-        s->T = static_cast<unsigned long long>(num >> 24);
-        s->above = 0;
-        s->prefix = 0;
-        if (s->T == 0) {
-          s->resolved = 1;
-          s->tb = s->maxbits;
-          s->need = 1;
-          done = 1;
-        }
-      }
-    }
-  }
+  if (threadIdx.x == 0) is_last = (atomicAdd(&s->arrived, 1u) == gridDim.x - 1);
   __syncthreads();
-  if (done) return;
-  const unsigned long long T = s->T;
-  const unsigned long long above = s->above;
-  // largest digit t with above + suf[t] >= T (exists: suf[0] covers everything not above)
-  const bool ok_here = above + suf[t] >= T;
-  const bool ok_next = (t + 1 < kBins) && (above + suf[t + 1] >= T);
-  __syncthreads();
-  if (ok_here && !ok_next) {
-    s->above = above + ((t + 1 < kBins) ? suf[t + 1] : 0ull);
-    s->prefix = (s->prefix << kDigitBits) | static_cast<unsigned int>(t);
-    if (pass == 2) {
-      const unsigned int tb = s->prefix;
-      s->tb = tb;
-      const unsigned long long ww = fixed_weight(tb);
-      const unsigned long long rest = T - s->above;
-      s->need = static_cast<unsigned int>((rest + ww - 1) / ww);
-      s->resolved = 1;
-    }
-  }
+  if (!is_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) s->arrived = 0;       // for the next pass
+  find_digit(pass, Pfix, keep_all, gh, s, status);
 }
 
 // Ties (bits == tb) per query-block row.  One warp per row.
@@ -461,8 +479,7 @@ cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double
   const int keep_all = p >= 1.0 ? 1 : 0;
   const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
   for (int pass = 0; pass < 3; ++pass) {
-    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
-    head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, bs->status);
+    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, P, keep_all, hist, st, bs->status);
   }
   const long long rows = static_cast<long long>(G) * nB;
   const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
@@ -564,8 +581,7 @@ extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t 
   const int keep_all = p >= 1.0 ? 1 : 0;
   const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
   for (int pass = 0; pass < 3; ++pass) {
-    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, hist, st);
-    head_find_kernel<<<G, kBins, 0, s>>>(pass, P, keep_all, hist, st, status);
+    head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, P, keep_all, hist, st, status);
   }
   const long long rows = static_cast<long long>(G) * nB;
   const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
