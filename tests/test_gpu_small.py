@@ -121,6 +121,32 @@ def test_bf16_pipeline(case, p):
     assert np.max(np.abs(host(lse) - ref_l[:, :, :wl.n_valid])) <= 1e-2
 
 
+@pytest.mark.parametrize("mode,scope,p", [("exact", "row", 0.9), ("meanpool", "head", 0.25)])
+def test_token_major_views_match_contiguous(mode, scope, p):
+    """[B, N, H, d] storage seen as [B, H, N, d] views (strided heads and rows):
+    every stage reads and writes through the strides, bit for bit as on copies."""
+    wl = small_workload("strided", 2, 3, 128, (3, 8, 12), 64, dtype="bf16", wid=130)
+    q, k, v = (x.cuda() for x in make_qkv(wl))
+    qs, ks, vs = (x.transpose(1, 2).contiguous().transpose(1, 2) for x in (q, k, v))
+    assert qs.stride(2) == wl.H * wl.d and not qs.is_contiguous()
+    perm = lbsa.lbsa_partition_perm(*wl.grid, "3d", device="cuda")
+    outs = []
+    for a, b_, c in ((q, k, v), (qs, ks, vs)):
+        ap, bp, cp = lbsa.lbsa_permute([a, b_, c], perm)
+        sc = lbsa.lbsa_score(ap, bp, wl.block, mode=mode)
+        bs = lbsa.lbsa_select(sc, wl.block, p, scope)
+        o = lbsa.lbsa_attend(ap, bp, cp, bs)
+        back = lbsa.lbsa_permute([o], perm, inverse=True)[0]
+        torch.cuda.synchronize()
+        assert lbsa.lbsa_device_status() == 0 and lbsa.lbsa_get_status(bs) == 0
+        outs.append((ap, sc, gpu_csr(bs), o, back))
+    (a0, s0, c0, o0, b0), (a1, s1, c1, o1, b1) = outs
+    assert torch.equal(a0, a1)
+    assert torch.equal(s0, s1)
+    assert_csr_equal(c1, c0)
+    assert torch.equal(o0, o1) and torch.equal(b0, b1)
+
+
 @pytest.mark.parametrize("case", BF16_CASES[:3], ids=lambda c: c[0])
 def test_bf16_dense_p1_equals_dense_attention(case):
     name, B, H, d, grid, block = case
