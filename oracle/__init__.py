@@ -8,11 +8,14 @@ computes, written from the pages' prose:
     smallest key/value block set whose retained mass meets a 99% threshold;
     the frozen block indices reused at later steps.
   * VMoBA (pith.science review of arXiv 2506.23858, "What carries the
-    argument", referee report major comment 1, circularity check, free
+    argument", referee report major comments 1-2, circularity check, free
     parameters): key blocks represented by their mean; global selection over
     all query-key block pairs of a head; threshold selection keeping the
     smallest number of pairs whose cumulative normalized similarity reaches
-    tau; the layer-wise 1D-2D-3D block partition; empty query rows.
+    tau; the layer-wise 1D-2D-3D block partition; empty query rows; the
+    "Local + TopK" selection of the training-free experiments.
+  * SCOPE (abstract, mlsift.com): hybrid Top-p with a head-specific Top-k
+    floor from the size-weighted mean of the initially retained counts.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It imports nothing from the CUDA library or its
@@ -22,6 +25,8 @@ Modules
   attention   dense_attention, sparse_attention        (pinned)
   scores      block_mass, meanpool_scores              (pinned)
   select      select_contract, select_fp64, csr tools  (pinned)
+  select_variants  select_local_topk (VMoBA "Local + TopK"), select_topp_floor
+              (SCOPE-style per-head floor over row top-p)   (pinned)
   partition   raster / 1D / 2D / 3D token orders       (pinned)
 
 Every function is pinned by a ``-m "not gpu"`` test against something other
@@ -32,13 +37,14 @@ from .attention import dense_attention, sparse_attention
 from .scores import block_mass, meanpool_scores
 from .select import (select_contract, select_fp64, InvalidScores, threshold_fixed_point,
                      csr_rows, csr_from_rows)
+from .select_variants import select_local_topk, select_topp_floor, floor_of_head
 from .partition import (perm_raster, perm_1d_temporal, perm_2d_frame_tiles, perm_3d_tiles,
                         perm_for_call, PARTITION_CYCLE)
 
 __all__ = [
     "dense_attention", "sparse_attention", "block_mass", "meanpool_scores",
     "select_contract", "select_fp64", "InvalidScores", "threshold_fixed_point",
-    "csr_rows", "csr_from_rows",
+    "csr_rows", "csr_from_rows", "select_local_topk", "select_topp_floor", "floor_of_head",
     "perm_raster", "perm_1d_temporal", "perm_2d_frame_tiles", "perm_3d_tiles",
     "perm_for_call", "PARTITION_CYCLE",
 ]
