@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
-    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2",
+    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule",
     "lbsa_select_head_noalloc", "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
@@ -72,6 +72,7 @@ def load_library():
     sig = {
         "lbsa_score": (ctypes.c_int, [P, P, ctypes.POINTER(_Desc), I32, I32, P, P, P]),
         "lbsa_select": (ctypes.c_int, [P, I32, I32, I32, I32, D, I32, ctypes.POINTER(P), P]),
+        "lbsa_select_rule": (ctypes.c_int, [P, I32, I32, I32, I32, I32, I32, D, I32, ctypes.POINTER(P), P]),
         "lbsa_attend": (ctypes.c_int, [P, P, P, ctypes.POINTER(_Desc), P, P, P, P]),
         "lbsa_free": (None, [P]),
         "lbsa_blockset_info": (ctypes.c_int, [P] + [ctypes.POINTER(I32)] * 5),
@@ -180,6 +181,26 @@ def lbsa_select(scores, block: int, p: float = 0.99, scope: str = "row", stream=
     h = ctypes.c_void_p()
     _check(load_library().lbsa_select(_ptr(scores), B, H, nB, block, float(p), _SCOPES[scope],
                                       ctypes.byref(h), _stream(stream)))
+    return Blockset(h.value)
+
+
+_RULES = {"local_topk": 0, "topp_floor": 1}
+
+
+def lbsa_select_rule(scores, block: int, rule: str, n_valid: int, p: float = 0.99, k: int = 0,
+                     stream=None) -> Blockset:
+    """Selection by a further rule into a new blockset (row scope): "local_topk"
+    keeps each row's own key block plus the k top-ranked others; "topp_floor"
+    applies the row threshold rule with p, then raises every row to its head's
+    size-weighted mean count (rounded up)."""
+    if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, nB, nB] tensor")
+    B, H, nB, nB2 = scores.shape
+    if nB != nB2:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be square per head")
+    h = ctypes.c_void_p()
+    _check(load_library().lbsa_select_rule(_ptr(scores), B, H, nB, block, int(n_valid), _RULES[rule], float(p),
+                                           int(k), ctypes.byref(h), _stream(stream)))
     return Blockset(h.value)
 
 

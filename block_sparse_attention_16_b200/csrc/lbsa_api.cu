@@ -266,6 +266,53 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
   return LBSA_OK;
 }
 
+int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, int32_t n_valid,
+                     int32_t rule, double p, int32_t k, lbsa_blockset** out, void* stream) {
+  int rc;
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if (B < 1 || H < 1 || nB < 1) return fail(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "the rank rules are built for nB <= 1024");
+  if (static_cast<long long>(nB - 1) * block >= n_valid || n_valid > static_cast<long long>(nB) * block)
+    return fail(LBSA_ERR_INVALID_ARG, "n_valid %d does not match nB %d x block %d", n_valid, nB, block);
+  if (rule == LBSA_RULE_LOCAL_TOPK) {
+    if (k < 0) return fail(LBSA_ERR_INVALID_ARG, "k = %d < 0", k);
+  } else if (rule == LBSA_RULE_TOPP_FLOOR) {
+    if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
+  } else {
+    return fail(LBSA_ERR_INVALID_ARG, "rule %d", rule);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  if ((rc = new_blockset(B, H, nB, block, LBSA_SCOPE_ROW, rule == LBSA_RULE_TOPP_FLOOR ? p : 0.0, s, &bs)) != LBSA_OK)
+    return rc;
+  const int R = B * H * nB;
+  cudaError_t e;
+  if (rule == LBSA_RULE_LOCAL_TOPK) {
+    e = lbsa::launch_select_rank(scores, R, nB, 0, k, nullptr, bs, s);
+  } else {
+    DeviceState* ds = nullptr;
+    Scratch ws;
+    if ((rc = device_state(&ds)) != LBSA_OK ||
+        (rc = scratch_alloc(ds, static_cast<size_t>(B) * H * sizeof(int32_t) + 256, s, &ws)) != LBSA_OK) {
+      lbsa_free(bs);
+      return rc;
+    }
+    int32_t* floor_dev = static_cast<int32_t*>(ws.ptr);
+    e = lbsa::launch_select_row(scores, R, nB, p, bs, s);
+    if (e == cudaSuccess) e = lbsa::launch_head_floor(bs->counts, B * H, nB, block, n_valid, floor_dev, s);
+    if (e == cudaSuccess) e = lbsa::launch_select_rank(scores, R, nB, 1, 0, floor_dev, bs, s);
+  }
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_select_rule launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
 int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, const lbsa_blockset* bs,
                 void* out, float* lse, void* stream) {
   int rc;

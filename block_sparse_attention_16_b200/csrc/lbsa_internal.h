@@ -65,6 +65,10 @@ cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d
 // selection (select.cu)
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,
                               cudaStream_t s);
+cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int k, const int32_t* head_floor,
+                               lbsa_blockset* bs, cudaStream_t s);
+cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, int n_valid, int32_t* head_floor,
+                              cudaStream_t s);
 size_t select_head_workspace_bytes(int B, int H, int nB);
 cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs,
                                void* workspace, cudaStream_t s);

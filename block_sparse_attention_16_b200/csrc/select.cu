@@ -439,6 +439,129 @@ inline uint32_t fixed_p(double p) {
   return static_cast<uint32_t>(std::nearbyint(p * 16777216.0));   // ties to even in the default mode
 }
 
+// ---------------------------------------------------------------- rank rules
+// Top-n of a row by rank (score bits descending, then lower id): one warp per
+// row, lane l holds ids l, l+32, ...; a 30-step bisection on the bits with
+// element counts finds the bits tb of the n-th ranked eligible element.
+//   mode 0 (Local + TopK, VMoBA review, referee report major comment 2): the
+//           row's own key block i = row % nB is kept and not ranked; n = k.
+//   mode 1 (top-p with a per-head floor, SCOPE abstract): n = max(c, min(K, nB))
+//           with c the threshold rule's count (already in the blockset) and K
+//           the head's floor; rows with n == c are left as they are.
+template <int EPL>
+__global__ void __launch_bounds__(256) select_rank_kernel(const float* __restrict__ scores, int R, int nB, int mode,
+                                                          int k, const int32_t* __restrict__ head_floor,
+                                                          int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+                                                          int32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;                       // warp-uniform
+  const int diag = (mode == 0) ? static_cast<int>(row % nB) : -1;
+  int n;
+  if (mode == 0) {
+    n = min(k, nB - 1);
+  } else {
+    const int c = counts[row];
+    n = max(c, min(head_floor[row / nB], nB));
+    if (n == c) return;
+  }
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
+  int32_t* out = cols + row * nB;
+  uint32_t bits[EPL];
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int idx = e * 32 + lane;
+    bits[e] = (idx < nB) ? __ldg(x + idx) : 0u;
+    bad |= (idx < nB) && (bits[e] >= kInvalidBits);
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) raise_status(status, LBSA_ERR_INVALID_SCORES);
+    for (int idx = lane; idx < nB; idx += 32) out[idx] = idx;
+    if (lane == 0) counts[row] = nB;
+    return;
+  }
+  uint32_t tb = 0u;                           // with n == 0 nothing is ranked in
+  uint32_t need = 0u;
+  if (n > 0) {
+    uint32_t lo = 0, hi = kInvalidBits;       // invariant: cnt(bits >= lo) >= n > cnt(bits >= hi)
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      uint32_t c = 0;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int idx = e * 32 + lane;
+        c += (idx < nB && idx != diag && bits[e] >= mid) ? 1u : 0u;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+      if (c >= static_cast<uint32_t>(n)) lo = mid;
+      else hi = mid;
+    }
+    tb = lo;
+    uint32_t above = 0;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int idx = e * 32 + lane;
+      above += (idx < nB && idx != diag && bits[e] > tb) ? 1u : 0u;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    need = static_cast<uint32_t>(n) - above;
+  }
+  // emit in ascending id order: the own block (mode 0), the ids ranked above tb,
+  // and the first `need` ties at tb in id order
+  int base = 0;
+  uint32_t ties_before = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int idx = e * 32 + lane;
+    const bool elig = idx < nB && idx != diag;
+    const bool tie = n > 0 && elig && bits[e] == tb;
+    const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+    const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+    const bool keep = (idx == diag) || (n > 0 && elig && (bits[e] > tb || (tie && rank < need)));
+    const uint32_t kmask = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[base + __popc(kmask & lt_mask)] = idx;
+    base += __popc(kmask);
+    ties_before += __popc(tmask);
+  }
+  if (lane == 0) counts[row] = base;
+}
+
+// One CTA of 256 threads per head: floor K = ceil(sum_i v_i c_i / sum_i v_i),
+// v_i = valid tokens of query block i, in exact integers.
+__global__ void __launch_bounds__(256) head_floor_kernel(const int32_t* __restrict__ counts, int nB, int block,
+                                                         int n_valid, int32_t* __restrict__ head_floor) {
+  __shared__ unsigned long long red[2][8];
+  const int g = blockIdx.x, lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  unsigned long long num = 0, den = 0;
+  for (int i = threadIdx.x; i < nB; i += blockDim.x) {
+    const unsigned long long v = static_cast<unsigned long long>(min(block, n_valid - i * block));
+    num += v * static_cast<unsigned long long>(counts[static_cast<long long>(g) * nB + i]);
+    den += v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    num += __shfl_xor_sync(0xffffffffu, num, o);
+    den += __shfl_xor_sync(0xffffffffu, den, o);
+  }
+  if (lane == 0) {
+    red[0][w] = num;
+    red[1][w] = den;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long N = 0, D = 0;
+    for (int u = 0; u < 8; ++u) {
+      N += red[0][u];
+      D += red[1][u];
+    }
+    head_floor[g] = static_cast<int32_t>((N + D - 1) / D);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s) {
@@ -457,6 +580,30 @@ cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa
   else if (nB <= 1024) LBSA_SEL(32);
   else return cudaErrorInvalidValue;
 #undef LBSA_SEL
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int k, const int32_t* head_floor,
+                               lbsa_blockset* bs, cudaStream_t s) {
+  const int threads = 256;
+  dim3 grid(static_cast<unsigned>((static_cast<long long>(R) * 32 + threads - 1) / threads));
+#define LBSA_RANK(EPL)                                                                                     \
+  select_rank_kernel<EPL><<<grid, threads, 0, s>>>(scores, R, nB, mode, k, head_floor, bs->counts, bs->cols, \
+                                                   bs->status)
+  if (nB <= 32) LBSA_RANK(1);
+  else if (nB <= 64) LBSA_RANK(2);
+  else if (nB <= 128) LBSA_RANK(4);
+  else if (nB <= 256) LBSA_RANK(8);
+  else if (nB <= 512) LBSA_RANK(16);
+  else if (nB <= 1024) LBSA_RANK(32);
+  else return cudaErrorInvalidValue;
+#undef LBSA_RANK
+  return cudaGetLastError();
+}
+
+cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, int n_valid, int32_t* head_floor,
+                              cudaStream_t s) {
+  head_floor_kernel<<<G, 256, 0, s>>>(counts, nB, block, n_valid, head_floor);
   return cudaGetLastError();
 }
 

@@ -101,7 +101,9 @@ typedef struct lbsa_blockset lbsa_blockset;
  *   lse     optional out (exact mode only; NULL to skip): fp32 [B, H, N_valid]
  *           contiguous, natural-log log-sum-exp of each query row of the dense
  *           pass.
- * The exact mode is a two-sweep dense pass (tensor cores for bf16). */
+ * The exact mode is one dense sweep (tensor cores for bf16) that keeps each
+ * row's per-chunk log-sum-exp and turns it into masses once the row's lse is
+ * known. */
 int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t block,
                int32_t mode, float* scores, float* lse, void* stream);
 
@@ -126,6 +128,28 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
  * stream-ordered at worst-case size (B*H*nB*(nB+1) int32); no host sync. */
 int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,
                 int32_t scope, lbsa_blockset** out, void* stream);
+
+/* Stage 2, two further rules of the pages, into a new blockset (row scope).
+ *   LBSA_RULE_LOCAL_TOPK  VMoBA review (referee report major comment 2: the
+ *       training-free experiments select blocks by "Local + TopK", with
+ *       k = 2, 6 or 18).  Row (b, h, i) keeps its own key block i plus the k
+ *       top-ranked other key blocks: min(k + 1, nB) blocks.  p, n_valid unused.
+ *   LBSA_RULE_TOPP_FLOOR  SCOPE abstract (a head-specific Top-k from the
+ *       query-size-weighted mean of the initially retained key counts; extra
+ *       keys only where the initial count falls below it).  The
+ *       LBSA_SCOPE_ROW threshold rule with p gives counts c_i; the head's
+ *       floor is K = ceil(sum_i v_i c_i / sum_i v_i) with v_i the valid tokens
+ *       of query block i, min(block, n_valid - i * block); row i keeps the
+ *       first max(c_i, min(K, nB)) blocks of its ranked order.  k unused.
+ * Ranked order: score descending, then key-block id ascending.  nB <= 1024.
+ * Invalid scores are handled as by lbsa_select.
+ *   n_valid  valid tokens: (nB - 1) * block < n_valid <= nB * block
+ *   p        in (0, 1] (LBSA_RULE_TOPP_FLOOR)
+ *   k        >= 0 (LBSA_RULE_LOCAL_TOPK)
+ *   out      receives a new blockset (free with lbsa_free). */
+typedef enum { LBSA_RULE_LOCAL_TOPK = 0, LBSA_RULE_TOPP_FLOOR = 1 } lbsa_rule;
+int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, int32_t n_valid,
+                     int32_t rule, double p, int32_t k, lbsa_blockset** out, void* stream);
 
 /* Stage 3: block-sparse attention over a (frozen) blockset.
  * VMoBA review "What carries the argument" (only selected blocks contribute
