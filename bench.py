@@ -544,6 +544,17 @@ def run_sweep(args):
         emit(workload="wan_skew", stage="attend", p=p, density=float(m.mean()),
              density_per_head=[round(float(x), 4) for x in m.mean(axis=(1, 2))], **ta, **tfl(fl, ta["median"]),
              select_ms=ts["median"])
+    # the two further rules on the same scores: SCOPE-style floor over row top-p,
+    # and VMoBA's Local + TopK at the pages' k values
+    rules = [("topp_floor", dict(p=p_)) for p_ in (0.9, 0.99)] + [("local_topk", dict(k=k_)) for k_ in (2, 6, 18)]
+    for rule, kw in rules:
+        bs = lbsa.lbsa_select_rule(sc, wl.block, rule, n_valid=wl.n_valid, **kw)
+        fl, m = flops_of(bs, wl)
+        ta = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+        ts = _timer(lambda: lbsa.lbsa_select_rule(sc, wl.block, rule, n_valid=wl.n_valid, **kw), flush=flush)
+        emit(workload="wan_skew", stage="attend", rule=rule, **kw, density=float(m.mean()),
+             density_per_head=[round(float(x), 4) for x in m.mean(axis=(1, 2))], **ta, **tfl(fl, ta["median"]),
+             select_ms=ts["median"], **{"select_" + k2: v2 for k2, v2 in hbm(sc.numel() * 4, ts["median"]).items()})
     del q, k, v, qp, kp, vp, sc
 
     # proxy mode: 1D / 2D / 3D cycle, head-scope selection at tau = 0.25

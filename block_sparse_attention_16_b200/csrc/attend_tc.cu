@@ -130,8 +130,20 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     tmem_alloc(misc, kTmemCols);
     tmem_relinquish();
   }
-  for (int i = tid; i < 2 * kMaxWords; i += kThreads) bm0[i] = 0;
+  for (int i = tid; i < nwords; i += kThreads) {
+    bm0[i] = 0;
+    bm1[i] = 0;
+  }
   __syncthreads();
+  if (warp == 4 && lane == 0) {
+    // the Q tile does not depend on the schedule: its load overlaps the build
+    prefetch_tmap(&tmap_q);
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+    mbar_arrive_expect_tx(bars.q_full, L::Q_BYTES);
+    for (int c = 0; c < D / 64; ++c)
+      tma_load_4d(smem + L::OFF_Q + c * BM * 128, &tmap_q, bars.q_full, c * 64, tile * BM, h, bb);
+  }
 
   const int qb0 = (blk == 64) ? 2 * tile : tile;
   const int qb1 = (blk == 64 && 2 * tile + 1 < nB) ? 2 * tile + 1 : -1;
@@ -191,14 +203,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tmap_q);
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
-      uint8_t* sQ = smem + L::OFF_Q;
-      if (n_steps > 0) {
-        mbar_arrive_expect_tx(bars.q_full, L::Q_BYTES);
-        for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, bars.q_full, c * 64, tile * BM, h, bb);
-      }
+      // a tile without steps never waits for Q: let the copy land before exit
+      if (n_steps == 0) mbar_wait(bars.q_full, 0, wl, args.status, nullptr);
       // K and V stream through separate rings: K stage s is free once S = Q K^T
       // of step s - NS has completed, V stage s once O += P V of step s - NS
       // has.  Both slots are probed without blocking so that a K load never
@@ -238,6 +244,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       }
       if (*abort_flag) {
         // let copies still in flight land before the CTA can exit
+        mbar_wait(bars.q_full, 0, wl, args.status, nullptr);
         for (int s = (sk > NS ? sk - NS : 0); s < sk; ++s) mbar_wait(bars.k_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
         for (int s = (sv > NS ? sv - NS : 0); s < sv; ++s) mbar_wait(bars.v_full + s % NS, (s / NS) & 1, wl, args.status, nullptr);
       }
