@@ -96,7 +96,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const int bb = blockIdx.z;
   const int nB = args.nB;
   const int blk = args.block;               // 64 or 128
-  const int spb = blk / BK;                 // steps per kept key block
+  const int spb_log = (blk == 128) ? 1 : 0;  // log2 of the steps per kept key block (no division in the loops)
+  const int spb = 1 << spb_log;
 
   Bars bars = make_bars(smem + L::OFF_BAR);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
@@ -219,8 +220,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         if (do_k || v_free) {
           const int s = do_k ? sk : sv;
           const int st = s % NS;
-          const uint32_t e = sched[s / spb];
-          const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
+          const uint32_t e = sched[s >> spb_log];
+          const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s & (spb - 1)) * BK;
           if (do_k) {
             uint8_t* sK = smem + L::OFF_K + st * L::KV_BYTES;
             mbar_arrive_expect_tx(bars.k_full + st, L::KV_BYTES);
@@ -309,8 +310,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const int sb = s & 1;
       if (!mbar_wait(bars.s_full + sb, (s >> 1) & 1, wl, args.status, abort_flag)) { alive = false; break; }
       tc_fence_after();
-      const uint32_t e = sched[s / spb];
-      const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s % spb) * BK;
+      const uint32_t e = sched[s >> spb_log];
+      const int key0 = static_cast<int>(e & 0xFFFFu) * blk + (s & (spb - 1)) * BK;
       const int nvk = args.N_valid - key0;     // valid keys in this step (may exceed 64)
       // warp-uniform: rows 0-63 (warps 0,1) and 64-127 (warps 2,3) are the two halves
       const bool take = (((e >> 30) >> half) & 1u) && nvk > 0;
