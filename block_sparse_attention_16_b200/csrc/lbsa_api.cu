@@ -212,7 +212,7 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
     if (desc->dtype == LBSA_BF16) {
       CUtensorMap tq, tk;
       if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
-      if ((rc = make_tmap(&tk, k, desc, 128)) != LBSA_OK) return rc;
+      if ((rc = make_tmap(&tk, k, desc, lbsa::score_exact_bf16_key_rows())) != LBSA_OK) return rc;
       if ((rc = scratch_alloc(ds, lbsa::score_exact_bf16_workspace_bytes(desc->B, desc->H, desc->N_valid), s, &ws)) !=
           LBSA_OK)
         return rc;

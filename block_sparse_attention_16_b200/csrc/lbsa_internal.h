@@ -50,6 +50,7 @@ cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, con
 cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
                                     cudaStream_t s);
 size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid);
+int score_exact_bf16_key_rows();   // rows of the K tensor map box the exact scorer loads per step
 
 // fp32 SIMT kernels (simt_f32.cu)
 cudaError_t launch_attend_f32(const float* q, const float* k, const float* v, const lbsa_qkv_desc& d,

@@ -14,22 +14,31 @@
 // partials are combined in a fixed order (deterministic).  Every Q K^T product
 // and every exponential of the dense pass is computed once.
 //
-// Persistent grid (two CTAs per SM, each walking tiles with a grid stride), so
-// the scratch is bounded: gridDim.x * (128 + 4) * n_chunks floats.  Each
+// Persistent grid (three CTAs per SM, each walking tiles with a grid stride),
+// so the scratch is bounded: gridDim.x * (128 + 4) * n_chunks floats.  Each
 // thread reads back only the strip values it wrote itself.
 //
 // Warp roles (192 threads): warps 0-3 softmax (thread t = tile row t = TMEM
-// lane t), warp 4 TMA producer (Q per tile, K 128-key tiles through a ring),
-// warp 5 UMMA issuer (S = Q K^T, M=128, N=128, K=d, double-buffered in TMEM
-// columns [0,128) and [128,256)).  One step covers two 64-key chunks; the
-// 128-wide UMMA keeps the tensor pipe's per-instruction cost amortised.
+// lane t), warp 4 TMA producer (Q per tile, K 64-key tiles through a 2-stage
+// ring), warp 5 UMMA issuer (S = Q K^T, M=128, N=64, K=d, double-buffered in
+// TMEM columns [0,64) and [64,128)).  About 67 KB of shared memory, 128 TMEM
+// columns and at most 112 registers a thread let three CTAs (three softmax
+// warps per SM sub-partition) share an SM, which hides more of the softmax's
+// dependent latency than two CTAs with 128-key steps.  The step width is a
+// build-time choice (LBSA_SCORE_BK = 64 or 128, LBSA_SCORE_CTAS = 3 or 2).
 #include "lbsa_device.cuh"
 
 namespace lbsa {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 128;           // keys per UMMA step
+#ifndef LBSA_SCORE_BK
+#define LBSA_SCORE_BK 64
+#endif
+#ifndef LBSA_SCORE_CTAS
+#define LBSA_SCORE_CTAS 3
+#endif
+constexpr int BK = LBSA_SCORE_BK;  // keys per UMMA step
 constexpr int CH = 64;            // keys per chunk (one mass entry per 64-key chunk)
 constexpr int NS = 2;
 // Of every 8 exponential pairs of a full chunk, those whose bit is set take
@@ -39,8 +48,8 @@ constexpr int NS = 2;
 #define LBSA_SCORE_POLY_MASK 0x88
 #endif
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 256;
-constexpr int kCtasPerSm = 2;
+constexpr uint32_t kTmemCols = 2 * BK;     // S double-buffered
+constexpr int kCtasPerSm = LBSA_SCORE_CTAS;
 template <int D>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
@@ -206,9 +215,9 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
           break;
         }
         tc_fence_after();
-        const int nh = min(2, n_chunks - 2 * j);      // chunks in this step (block-uniform)
+        const int nh = min(BK / CH, n_chunks - (BK / CH) * j);   // chunks in this step (block-uniform)
         for (int hf = 0; hf < nh; ++hf) {
-          const int ch = 2 * j + hf;
+          const int ch = (BK / CH) * j + hf;
           uint32_t r[64];
           tmem_ld32(t_lane + sb * BK + hf * CH, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           tmem_ld32(t_lane + sb * BK + hf * CH + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -340,6 +349,8 @@ int score_grid(int N, int H, int B) {
 }
 
 }  // namespace
+
+int score_exact_bf16_key_rows() { return BK; }
 
 size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid) {
   const int n_chunks = (N_valid + CH - 1) / CH;
