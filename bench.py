@@ -529,6 +529,11 @@ def run_sweep(args):
     emit(workload="wan", stage="attend_dense_p1", **t, **tfl(fld, t["median"]))
     t = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp))
     emit(workload="wan", stage="torch_sdpa_dense (library reference)", **t, **tfl(fld, t["median"]))
+    # the fused dense step: dense O and the exact block masses from one sweep
+    sc_f, o_f = lbsa.lbsa_score_attend(qp, kp, vp, wl.block)
+    t = _timer(lambda: lbsa.lbsa_score_attend(qp, kp, vp, wl.block, scores=sc_f, out=o_f))
+    emit(workload="wan", stage="fused_dense_step (dense O + exact masses)", **t, **tfl(fld, t["median"]))
+    del sc_f, o_f
     del q, k, v, qp, kp, vp, sc, bs, dense
 
     # skewed heads: p sweep

@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
-    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule",
+    "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule", "lbsa_score_attend",
     "lbsa_select_head_noalloc", "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
@@ -73,6 +73,7 @@ def load_library():
         "lbsa_score": (ctypes.c_int, [P, P, ctypes.POINTER(_Desc), I32, I32, P, P, P]),
         "lbsa_select": (ctypes.c_int, [P, I32, I32, I32, I32, D, I32, ctypes.POINTER(P), P]),
         "lbsa_select_rule": (ctypes.c_int, [P, I32, I32, I32, I32, I32, I32, D, I32, ctypes.POINTER(P), P]),
+        "lbsa_score_attend": (ctypes.c_int, [P, P, P, ctypes.POINTER(_Desc), I32, P, P, P, P]),
         "lbsa_attend": (ctypes.c_int, [P, P, P, ctypes.POINTER(_Desc), P, P, P, P]),
         "lbsa_free": (None, [P]),
         "lbsa_blockset_info": (ctypes.c_int, [P] + [ctypes.POINTER(I32)] * 5),
@@ -182,6 +183,28 @@ def lbsa_select(scores, block: int, p: float = 0.99, scope: str = "row", stream=
     _check(load_library().lbsa_select(_ptr(scores), B, H, nB, block, float(p), _SCOPES[scope],
                                       ctypes.byref(h), _stream(stream)))
     return Blockset(h.value)
+
+
+def lbsa_score_attend(q, k, v, block: int, scores=None, out=None, lse=None, want_lse=False, stream=None):
+    """Dense attention that also returns the exact block masses (one sweep).
+
+    Returns (scores [B, H, nB, nB] fp32, out) or (scores, out, lse)."""
+    _same_layout(q, k)
+    _same_layout(q, v)
+    B, H, N, _ = q.shape
+    nB = -(-N // block)
+    if scores is None:
+        scores = torch.empty(B, H, nB, nB, dtype=torch.float32, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _same_layout(q, out)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    desc = _desc(q)
+    _check(load_library().lbsa_score_attend(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(desc), block, _ptr(scores),
+                                            _ptr(out), _ptr(lse), _stream(stream)))
+    return (scores, out, lse) if want_lse else (scores, out)
 
 
 _RULES = {"local_topk": 0, "topp_floor": 1}

@@ -230,6 +230,41 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
   return LBSA_OK;
 }
 
+int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, int32_t block,
+                      float* scores, void* out, float* lse, void* stream) {
+  int rc;
+  if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(v, "v")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if ((rc = validate_ptr(out, "out")) != LBSA_OK) return rc;
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  if (desc->dtype != LBSA_BF16) return fail(LBSA_ERR_UNSUPPORTED, "the fused dense step is built for bf16");
+  const int nB = n_blocks(desc->N_valid, block);
+  if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "nB %d > 4096", nB);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != LBSA_OK) return rc;
+  int n_slots = 0;
+  size_t flag_bytes = 0;
+  const size_t bytes = lbsa::score_attend_bf16_workspace_bytes(desc->N_valid, &n_slots, &flag_bytes);
+  Scratch ws;
+  if ((rc = scratch_alloc(ds, bytes, s, &ws)) != LBSA_OK) return rc;
+  lbsa::AttendArgs a{desc->B, desc->H, desc->N_valid, desc->d, block, nB, nullptr, nullptr, ds->status,
+                     out, desc->stride_b, desc->stride_h, desc->stride_n, lse, wait_limit(),
+                     scores, reinterpret_cast<float*>(static_cast<char*>(ws.ptr) + flag_bytes),
+                     static_cast<int32_t*>(ws.ptr), n_slots};
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
+  if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
+  if ((rc = make_tmap(&tv, v, desc, 64)) != LBSA_OK) return rc;
+  cudaError_t e = cudaMemsetAsync(ws.ptr, 0, flag_bytes, s);     // every strip slot free
+  if (e == cudaSuccess) e = lbsa::launch_score_attend_bf16(&tq, &tk, &tv, a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_score_attend launch");
+  return LBSA_OK;
+}
+
 int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p, int32_t scope,
                 lbsa_blockset** out, void* stream) {
   int rc;

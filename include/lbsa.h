@@ -107,6 +107,21 @@ typedef struct lbsa_blockset lbsa_blockset;
 int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t block,
                int32_t mode, float* scores, float* lse, void* stream);
 
+/* Stages 1 and 3 fused for a dense step: dense attention that also returns
+ * the exact block masses of lbsa_score (LoSA abstract: the masses are measured
+ * at one early dense step; that step's attention output is needed anyway).
+ * One sweep over the keys: per 64-key chunk each row keeps its chunk
+ * log-sum-exp in a strip, the row's lse then turns the strip into masses.
+ *   q, k, v  bf16 [B, H, N_valid, d] per desc (fp32 returns LBSA_ERR_UNSUPPORTED)
+ *   block    64 or 128 (the mass granularity)
+ *   scores   out: fp32 [B, H, nB, nB] contiguous, as lbsa_score (exact mode)
+ *   out      out: dense attention output, same dtype and strides as q
+ *   lse      optional out: fp32 [B, H, N_valid] natural-log row log-sum-exp
+ * Scratch: (2 x SM count) strips of (128 + 4) x ceil(N_valid / 64) floats,
+ * from the library pool. */
+int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, int32_t block,
+                      float* scores, void* out, float* lse, void* stream);
+
 /* Stage 2: mass-threshold selection into a new blockset.
  * LoSA abstract (per head and query block, smallest set meeting the
  * threshold); VMoBA review (global selection over a head; threshold tau;
