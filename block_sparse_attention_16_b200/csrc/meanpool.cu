@@ -17,64 +17,117 @@ namespace {
 
 constexpr int kTile = 64;
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
-  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = __bfloat1622float2(h[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
+int g_sms = 0;
+int num_sms() {
+  if (!g_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms <= 0) g_sms = 148;
   }
-}
-__device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  return g_sms;
 }
 
-// grid (nB, H, B), 256 threads: thread = (row group g, 8-column vector v).
-template <typename T, int D>
-__global__ void block_mean_kernel(const T* __restrict__ q, const T* __restrict__ k, lbsa_qkv_desc desc, int block,
-                                  int nB, float* __restrict__ qbar, float* __restrict__ kbar) {
-  constexpr int V = D / 8;               // vectors per row
-  constexpr int G = 256 / V;             // row groups
-  __shared__ float red[2][G][D];
-  const int i = blockIdx.x, h = blockIdx.y, bb = blockIdx.z;
-  const int v = threadIdx.x % V, g = threadIdx.x / V;
-  const int r0 = i * block, r1 = min(r0 + block, desc.N_valid);
-  const long long base = bb * desc.stride_b + h * desc.stride_h;
-  float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  // at most 128 / G rows per thread: unrolled and predicated, so that all of a
-  // thread's 16-byte loads are in flight together
-  constexpr int kMaxIt = 128 / G;
+// Eight consecutive columns of one row as raw 16-byte vectors (one for bf16,
+// two for fp32), so that a thread's loads for a whole block can be issued
+// before any of them is used.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 a;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { a = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void add_to(float (&f)[8]) const {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&a);
 #pragma unroll
-  for (int it = 0; it < kMaxIt; ++it) {
-    const int r = r0 + g + it * G;
-    if (r < r1) {
-      float f[8];
-      load8(q + base + r * desc.stride_n + v * 8, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) aq[e] += f[e];
-      load8(k + base + r * desc.stride_n + v * 8, f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ak[e] += f[e];
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] += t.x;
+      f[2 * i + 1] += t.y;
     }
   }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    red[0][g][v * 8 + e] = aq[e];
-    red[1][g][v * 8 + e] = ak[e];
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
   }
-  __syncthreads();
-  const float inv = 1.0f / static_cast<float>(r1 - r0);
-  const long long o = ((static_cast<long long>(bb) * desc.H + h) * nB + i) * D;
-  for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
-    const int which = c / D, col = c % D;
-    float s = 0.f;
-    for (int gg = 0; gg < G; ++gg) s += red[which][gg][col];
-    (which ? kbar : qbar)[o + col] = s * inv;
+  __device__ __forceinline__ void add_to(float (&f)[8]) const {
+    f[0] += a.x; f[1] += a.y; f[2] += a.z; f[3] += a.w;
+    f[4] += b.x; f[5] += b.y; f[6] += b.z; f[7] += b.w;
+  }
+};
+
+// Persistent grid over the (b, h, block) items (blocks of at most MAXR
+// tokens), 256 threads: thread = (row group g, 8-column vector v).  The loads of a thread's next item are issued
+// before the current item's sums are reduced, so DRAM traffic continues
+// through the reduction.  Reduction: lanes of a warp that share v by
+// shuffles, then the eight warps through double-buffered shared memory (one
+// barrier per item).
+template <typename T, int D, int MAXR>
+__global__ void __launch_bounds__(256) block_mean_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                                                         lbsa_qkv_desc desc, int block, int nB, long long items,
+                                                         float* __restrict__ qbar, float* __restrict__ kbar) {
+  constexpr int V = D / 8;               // vectors per row
+  constexpr int G = 256 / V;             // row groups
+  constexpr int kMaxIt = MAXR / G;       // rows per thread at block = MAXR
+  __shared__ float red[2][8][2 * D];
+  const int v = threadIdx.x % V, g = threadIdx.x / V;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Raw8<T> rq[kMaxIt], rk[kMaxIt];
+  auto issue = [&](long long item) {
+    const int i = static_cast<int>(item % nB);
+    const long long bh = item / nB;
+    const int h = static_cast<int>(bh % desc.H), bb = static_cast<int>(bh / desc.H);
+    const int r0 = i * block, r1 = min(r0 + block, desc.N_valid);
+    const long long base = bb * desc.stride_b + h * desc.stride_h + v * 8;
+#pragma unroll
+    for (int it = 0; it < kMaxIt; ++it) {
+      const int r = r0 + g + it * G;
+      if (r < r1) {
+        rq[it].load(q + base + r * desc.stride_n);
+        rk[it].load(k + base + r * desc.stride_n);
+      }
+    }
+  };
+  long long item = blockIdx.x;
+  if (item < items) issue(item);
+  for (int buf = 0; item < items; item += gridDim.x, buf ^= 1) {
+    const int i = static_cast<int>(item % nB);
+    const int r0 = i * block, r1 = min(r0 + block, desc.N_valid);
+    float aq[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ak[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int it = 0; it < kMaxIt; ++it) {
+      if (r0 + g + it * G < r1) {
+        rq[it].add_to(aq);
+        rk[it].add_to(ak);
+      }
+    }
+    if (item + gridDim.x < items) issue(item + gridDim.x);
+#pragma unroll
+    for (int o = V; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        aq[e] += __shfl_xor_sync(0xffffffffu, aq[e], o);
+        ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], o);
+      }
+    if (lane < V) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        red[buf][warp][v * 8 + e] = aq[e];
+        red[buf][warp][D + v * 8 + e] = ak[e];
+      }
+    }
+    __syncthreads();
+    const float inv = 1.0f / static_cast<float>(r1 - r0);
+    for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[buf][w][c];
+      (c < D ? qbar : kbar)[item * D + (c % D)] = s * inv;
+    }
   }
 }
 
@@ -97,21 +150,32 @@ __global__ void __launch_bounds__(256) logits_kernel(const float* __restrict__ q
   const float* kb = kbar + static_cast<long long>(g) * nB * D;
   const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
   float acc[4][4] = {};
-  for (int c0 = 0; c0 < D; c0 += KC) {
-    // 64 rows x 8 float4 per operand: two float4 per thread per operand
+  // the next round's operands are fetched into registers while this round computes
+  float4 na[2], nb[2];
+  auto fetch = [&](int c0) {
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
       const int e = threadIdx.x + it * 256;
       const int r = e >> 3, c4 = (e & 7) * 4;
       const int qi = ti * kTile + r, kj = tj * kTile + r;
-      const float4 a = (qi < nB) ? *reinterpret_cast<const float4*>(qb + static_cast<long long>(qi) * D + c0 + c4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 b = (kj < nB) ? *reinterpret_cast<const float4*>(kb + static_cast<long long>(kj) * D + c0 + c4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      sq[c4][r] = a.x; sq[c4 + 1][r] = a.y; sq[c4 + 2][r] = a.z; sq[c4 + 3][r] = a.w;
-      sk[c4][r] = b.x; sk[c4 + 1][r] = b.y; sk[c4 + 2][r] = b.z; sk[c4 + 3][r] = b.w;
+      na[it] = (qi < nB) ? *reinterpret_cast<const float4*>(qb + static_cast<long long>(qi) * D + c0 + c4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+      nb[it] = (kj < nB) ? *reinterpret_cast<const float4*>(kb + static_cast<long long>(kj) * D + c0 + c4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  fetch(0);
+  for (int c0 = 0; c0 < D; c0 += KC) {
+    // 64 rows x 8 float4 per operand: two float4 per thread per operand, stored transposed
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int e = threadIdx.x + it * 256;
+      const int r = e >> 3, c4 = (e & 7) * 4;
+      sq[c4][r] = na[it].x; sq[c4 + 1][r] = na[it].y; sq[c4 + 2][r] = na[it].z; sq[c4 + 3][r] = na[it].w;
+      sk[c4][r] = nb[it].x; sk[c4 + 1][r] = nb[it].y; sk[c4 + 2][r] = nb[it].z; sk[c4 + 3][r] = nb[it].w;
     }
     __syncthreads();
+    if (c0 + KC < D) fetch(c0 + KC);
 #pragma unroll 8
     for (int c = 0; c < KC; ++c) {
       const float4 a = *reinterpret_cast<const float4*>(&sq[c][tr]);
@@ -193,6 +257,20 @@ __global__ void normalize_kernel(float* __restrict__ scores, const float2* __res
     s[i] = expf(s[i] - M) * invZ;
 }
 
+// One CTA per resident slot (persistent), from the occupancy of this instantiation.
+template <typename T, int D, int MAXR>
+void launch_mean(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, long long items,
+                 float* qbar, float* kbar, cudaStream_t s) {
+  static int per_sm = 0;
+  if (!per_sm) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_mean_kernel<T, D, MAXR>, 256, 0);
+    if (per_sm <= 0) per_sm = 1;
+  }
+  const unsigned grid = static_cast<unsigned>(std::min<long long>(items, static_cast<long long>(per_sm) * num_sms()));
+  block_mean_kernel<T, D, MAXR><<<grid, 256, 0, s>>>(static_cast<const T*>(q), static_cast<const T*>(k), d, block,
+                                                     nB, items, qbar, kbar);
+}
+
 template <int D>
 cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, float* scores, void* ws,
                 cudaStream_t s) {
@@ -201,13 +279,18 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
   float* kbar = qbar + G * nB * D;
   float2* part = reinterpret_cast<float2*>(kbar + G * nB * D);
   const int nT = (nB + kTile - 1) / kTile;
-  if (d.dtype == LBSA_BF16)
-    block_mean_kernel<__nv_bfloat16, D><<<dim3(nB, d.H, d.B), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), d, block, nB, qbar, kbar);
-  else
-    block_mean_kernel<float, D><<<dim3(nB, d.H, d.B), 256, 0, s>>>(static_cast<const float*>(q),
-                                                                    static_cast<const float*>(k), d, block, nB,
-                                                                    qbar, kbar);
+  const long long items = G * nB;
+  if (d.dtype == LBSA_BF16) {
+    if (block <= 64)
+      launch_mean<__nv_bfloat16, D, 64>(q, k, d, block, nB, items, qbar, kbar, s);
+    else
+      launch_mean<__nv_bfloat16, D, 128>(q, k, d, block, nB, items, qbar, kbar, s);
+  } else {
+    if (block <= 64)
+      launch_mean<float, D, 64>(q, k, d, block, nB, items, qbar, kbar, s);
+    else
+      launch_mean<float, D, 128>(q, k, d, block, nB, items, qbar, kbar, s);
+  }
   logits_kernel<D><<<dim3(nT, nT, static_cast<unsigned>(G)), 256, 0, s>>>(
       qbar, kbar, nB, static_cast<float>(1.0 / std::sqrt(static_cast<double>(D))), scores, part);
   const int chunks = static_cast<int>(std::min<long long>(64, (static_cast<long long>(nB) * nB + 2047) / 2048));

@@ -40,7 +40,10 @@ constexpr int BM = 128;
 #endif
 constexpr int BK = LBSA_SCORE_BK;  // keys per UMMA step
 constexpr int CH = 64;            // keys per chunk (one mass entry per 64-key chunk)
-constexpr int NS = 2;
+#ifndef LBSA_SCORE_NS
+#define LBSA_SCORE_NS 2
+#endif
+constexpr int NS = LBSA_SCORE_NS;  // K ring depth
 // Of every 8 exponential pairs of a full chunk, those whose bit is set take
 // the FMA-pipe exponential (exp2_poly2) instead of MUFU ex2: a quarter of the
 // exponentials moves off the MUFU, which otherwise bounds the softmax warps.
@@ -136,6 +139,8 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
       prefetch_tmap(&tmap_k);
       uint8_t* sQ = smem + L::OFF_Q;
       long long s = 0;       // global step counter (ring position)
+      int st = 0;            // s % NS
+      uint32_t ph = 0;       // (s / NS) & 1
       int it = 0;            // tiles handled by this CTA
       bool ok = true;
       for (int g = blockIdx.x; ok && g < total_tiles; g += gridDim.x, ++it) {
@@ -144,14 +149,17 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
         mbar_arrive_expect_tx(q_full, L::Q_BYTES);
         for (int c = 0; c < D / 64; ++c) tma_load_4d(sQ + c * BM * 128, &tmap_q, q_full, c * 64, t.tile * BM, t.h, t.bb);
         for (int j = 0; j < n_steps; ++j, ++s) {
-          const int st = static_cast<int>(s % NS);
-          if (s >= NS && !mbar_wait(k_empty + st, static_cast<uint32_t>((s / NS) & 1) ^ 1u, wl, args.status, abort_flag)) {
+          if (s >= NS && !mbar_wait(k_empty + st, ph ^ 1u, wl, args.status, abort_flag)) {
             ok = false;
             break;
           }
           uint8_t* sK = smem + L::OFF_K + st * L::K_BYTES;
           mbar_arrive_expect_tx(k_full + st, L::K_BYTES);
           for (int c = 0; c < D / 64; ++c) tma_load_4d(sK + c * BK * 128, &tmap_k, k_full + st, c * 64, j * BK, t.h, t.bb);
+          if (++st == NS) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
       }
       if (*abort_flag) {
@@ -167,14 +175,15 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
       const uint32_t sQ = smem_u32(smem + L::OFF_Q);
       const uint32_t sK0 = smem_u32(smem + L::OFF_K);
       long long s = 0;
+      int st = 0;            // s % NS
+      uint32_t ph = 0;       // (s / NS) & 1
       int it = 0;
       bool ok = true;
       for (int g = blockIdx.x; ok && g < total_tiles; g += gridDim.x, ++it) {
         if (!mbar_wait(q_full, it & 1, wl, args.status, abort_flag)) break;
         for (int j = 0; j < n_steps; ++j, ++s) {
-          const int st = static_cast<int>(s % NS);
           const int sb = static_cast<int>(s & 1);
-          if (!mbar_wait(k_full + st, static_cast<uint32_t>((s / NS) & 1), wl, args.status, abort_flag) ||
+          if (!mbar_wait(k_full + st, ph, wl, args.status, abort_flag) ||
               (s >= 2 && !mbar_wait(s_free + sb, static_cast<uint32_t>(((s - 2) >> 1) & 1), wl, args.status, abort_flag))) {
             ok = false;
             break;
@@ -190,6 +199,10 @@ score_exact_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid
           }
           umma_commit(s_full + sb);
           umma_commit(k_empty + st);
+          if (++st == NS) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
         umma_commit(q_empty);          // Q may be replaced once this tile's UMMAs are done
       }

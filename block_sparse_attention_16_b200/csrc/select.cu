@@ -95,10 +95,11 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
     uint32_t lo = 0, hi = kInvalidBits;       // invariant: S(lo) >= T > S(hi)
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
-      uint64_t s = 0;
+      // four independent partial sums: the 64-bit adds do not form one long chain
+      uint64_t s4[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) s += (bits[e] >= mid) ? w[e] : 0;
-      s = warp_sum_u64(s);
+      for (int e = 0; e < EPL; ++e) s4[e & 3] += (bits[e] >= mid) ? w[e] : 0;
+      const uint64_t s = warp_sum_u64((s4[0] + s4[1]) + (s4[2] + s4[3]));
       if (s >= T) lo = mid;
       else hi = mid;
     }
@@ -567,7 +568,9 @@ __global__ void __launch_bounds__(256) head_floor_kernel(const int32_t* __restri
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s) {
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  const int threads = 256;
+  // two warps (rows) per block: residency is then bounded by registers, not by
+  // the block granularity of the register-heavy wide-row instantiations
+  const int threads = 64;
   const long long blocks = (static_cast<long long>(R) * 32 + threads - 1) / threads;
   dim3 grid(static_cast<unsigned>(blocks));
 #define LBSA_SEL(EPL)                                                                                       \
