@@ -194,6 +194,44 @@ def test_hand_built_lists_with_empty_rows(dtype, block):
     assert np.all(host(out)[empty] == 0)
 
 
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_running_max_rescales_within_and_across_steps(block):
+    """Logits that climb steeply along the key axis (head 0) make the running
+    max grow inside a 128-key step and at every step, so P already written and
+    O are rescaled; falling logits (head 1) never rescale after the first key.
+    Dense lists and random lists with empty rows, against the fp64 oracle."""
+    B, H, d, n_valid = 1, 2, 128, 600            # 10 (b=64) or 5 (b=128) blocks, ragged last block
+    nB = (n_valid + block - 1) // block
+    g = torch.Generator().manual_seed(140 + block)
+    q = torch.randn(B, H, n_valid, d, generator=g) * 0.5
+    k = torch.randn(B, H, n_valid, d, generator=g) * 0.5
+    v = torch.randn(B, H, n_valid, d, generator=g)
+    ramp = torch.arange(n_valid, dtype=torch.float32) * 0.35 * (d ** 0.5) / (8.0 * 1.4426950408889634)
+    q[:, :, :, 0] = 8.0
+    k[0, 0, :, 0] = ramp                          # +0.35 per key in log2 units: +22 over a 64-key half
+    k[0, 1, :, 0] = ramp.flip(0)
+    q, k, v = (x.to(torch.bfloat16).cuda() for x in (q, k, v))
+    rng = np.random.default_rng(block)
+    dense = [np.arange(nB) for _ in range(B * H * nB)]
+    sparse = []
+    for _ in range(B * H * nB):
+        r = rng.random()
+        sparse.append(np.zeros(0, dtype=np.int64) if r < 0.2 else
+                      np.sort(rng.choice(nB, size=int(rng.integers(1, nB + 1)), replace=False)))
+    for rows in (dense, sparse):
+        rp, col = oracle.csr_from_rows(rows)
+        bs = lbsa.lbsa_blockset_from_csr(torch.from_numpy(rp).cuda(), torch.from_numpy(col).cuda(), B, H, nB, block)
+        out, lse = lbsa.lbsa_attend(q, k, v, bs, want_lse=True)
+        torch.cuda.synchronize()
+        assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+        ref_o, ref_l = oracle.sparse_attention(host(q), host(k), host(v), n_valid, block, rp, col)
+        assert_out_close(host(out), ref_o[:, :, :n_valid], torch.bfloat16)
+        gl, rl = host(lse), ref_l[:, :, :n_valid]
+        assert np.array_equal(np.isneginf(gl), np.isneginf(rl))
+        fin = np.isfinite(rl)
+        assert np.max(np.abs(gl[fin] - rl[fin])) <= 1e-2
+
 def test_bad_block_index_is_flagged_and_skipped():
     wl = small_workload("bad", 1, 1, 128, (2, 8, 16), 64, dtype="bf16", wid=131)   # 256 tokens, 4 blocks
     q, k, v = (x.cuda() for x in make_qkv(wl))
