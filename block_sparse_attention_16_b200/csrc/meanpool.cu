@@ -252,9 +252,36 @@ __global__ void normalize_kernel(float* __restrict__ scores, const float2* __res
   const float M = sM, invZ = 1.0f / sZ;
   const long long n = static_cast<long long>(nB) * nB;
   float* s = scores + static_cast<long long>(g) * n;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    s[i] = expf(s[i] - M) * invZ;
+  // 16-byte vectors (nB*nB is a multiple of 4 when nB is even), four in flight per thread
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if ((n & 3) == 0 && (reinterpret_cast<uintptr_t>(s) & 15) == 0) {
+    float4* s4 = reinterpret_cast<float4*>(s);
+    const long long n4 = n >> 2;
+    for (; i + 3 * stride < n4; i += 4 * stride) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = s4[i + u * stride];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[u].x = expf(v[u].x - M) * invZ;
+        v[u].y = expf(v[u].y - M) * invZ;
+        v[u].z = expf(v[u].z - M) * invZ;
+        v[u].w = expf(v[u].w - M) * invZ;
+        s4[i + u * stride] = v[u];
+      }
+    }
+    for (; i < n4; i += stride) {
+      float4 v = s4[i];
+      v.x = expf(v.x - M) * invZ;
+      v.y = expf(v.y - M) * invZ;
+      v.z = expf(v.z - M) * invZ;
+      v.w = expf(v.w - M) * invZ;
+      s4[i] = v;
+    }
+  } else {
+    for (; i < n; i += stride) s[i] = expf(s[i] - M) * invZ;
+  }
 }
 
 // One CTA per resident slot (persistent), from the occupancy of this instantiation.
