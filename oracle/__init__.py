@@ -9,8 +9,9 @@ computes, written from the pages' prose:
     the frozen block indices reused at later steps.
   * VMoBA (pith.science review of arXiv 2506.23858, "What carries the
     argument", referee report major comments 1-2, circularity check, free
-    parameters): key blocks represented by their mean; global selection over
-    all query-key block pairs of a head; threshold selection keeping the
+    parameters): key blocks represented by their mean, scored by query-block
+    means or by every query token; global selection over all query-key block
+    (or query-token, key-block) pairs of a head; threshold selection keeping the
     smallest number of pairs whose cumulative normalized similarity reaches
     tau; the layer-wise 1D-2D-3D block partition; empty query rows; the
     "Local + TopK" selection of the training-free experiments.
@@ -22,8 +23,8 @@ leg may import this package.  It imports nothing from the CUDA library or its
 Python binding and shares no helper with them.
 
 Modules
-  attention   dense_attention, sparse_attention        (pinned)
-  scores      block_mass, meanpool_scores              (pinned)
+  attention   dense_attention, sparse_attention, token_sparse_attention   (pinned)
+  scores      block_mass, meanpool_scores, token_meanpool_scores      (pinned)
   select      select_contract, select_fp64, csr tools  (pinned)
   select_variants  select_local_topk (VMoBA "Local + TopK"), select_topp_floor
               (SCOPE-style per-head floor over row top-p)   (pinned)
@@ -33,8 +34,8 @@ Every function is pinned by a ``-m "not gpu"`` test against something other
 than itself (library routines, closed forms, brute force, hand-worked
 examples under ``tests/golden/``); none is "parity unpinned".
 """
-from .attention import dense_attention, sparse_attention
-from .scores import block_mass, meanpool_scores
+from .attention import dense_attention, sparse_attention, token_sparse_attention
+from .scores import block_mass, meanpool_scores, token_meanpool_scores
 from .select import (select_contract, select_fp64, InvalidScores, threshold_fixed_point,
                      csr_rows, csr_from_rows)
 from .select_variants import select_local_topk, select_topp_floor, floor_of_head
@@ -42,7 +43,8 @@ from .partition import (perm_raster, perm_1d_temporal, perm_2d_frame_tiles, perm
                         perm_for_call, PARTITION_CYCLE)
 
 __all__ = [
-    "dense_attention", "sparse_attention", "block_mass", "meanpool_scores",
+    "dense_attention", "sparse_attention", "token_sparse_attention", "block_mass", "meanpool_scores",
+    "token_meanpool_scores",
     "select_contract", "select_fp64", "InvalidScores", "threshold_fixed_point",
     "csr_rows", "csr_from_rows", "select_local_topk", "select_topp_floor", "floor_of_head",
     "perm_raster", "perm_1d_temporal", "perm_2d_frame_tiles", "perm_3d_tiles",

@@ -22,6 +22,14 @@ block-granular reading used here scores the query-block mean instead:
 
 "normalized similarity" (review, circularity check) is read as this softmax
 over all query-block x key-block pairs of the head.
+
+token_meanpool_scores -- the same proxy in the pages' own granularity: every
+query token scores every key-block mean ("full query-by-block similarity
+matrix", referee report major comment 1), and the similarities of one head
+are normalised by a softmax over all of its (query token, key block) pairs:
+
+    s_rj = q_r . kbar_j / sqrt(d)      for valid tokens r < n_valid
+    score[b,h,r,j] = exp(s_rj) / sum_{r',j'} exp(s_r'j')   (over the head)
 """
 from __future__ import annotations
 
@@ -67,6 +75,22 @@ def meanpool_scores(q, k, n_valid: int, block: int):
             kbar = np.stack([k[b, h, j * block:min((j + 1) * block, n_valid)].mean(axis=0)
                              for j in range(nB)])
             s = (qbar @ kbar.T) / np.sqrt(d)
+            e = np.exp(s - s.max())
+            out[b, h] = e / e.sum()
+    return out
+
+
+def token_meanpool_scores(q, k, n_valid: int, block: int):
+    """Per-token proxy scores [B, H, n_valid, nB], softmax-normalised over each head."""
+    q, k = _f64(q), _f64(k)
+    B, H, _, d = q.shape
+    nB = -(-n_valid // block)
+    out = np.zeros((B, H, n_valid, nB))
+    for b in range(B):
+        for h in range(H):
+            kbar = np.stack([k[b, h, j * block:min((j + 1) * block, n_valid)].mean(axis=0)
+                             for j in range(nB)])
+            s = (q[b, h, :n_valid] @ kbar.T) / np.sqrt(d)
             e = np.exp(s - s.max())
             out[b, h] = e / e.sum()
     return out

@@ -22,8 +22,9 @@ Readings taken where the pages are silent:
   * Scores that are NaN, negative (sign bit set, -0.0 included) or >= 2 are
     rejected.
   * Scope "row": one segment per (b, h, query block); scope "head": one
-    segment per (b, h) over all nB*nB pairs, flat index i*nB + j.  Kept
-    columns are emitted per query-block row in ascending order (CSR).
+    segment per (b, h) over all nQ*nB pairs, flat index i*nB + j, where the
+    nQ rows are query blocks (block-mean proxy) or query tokens (per-token
+    proxy).  Kept columns are emitted per row in ascending order (CSR).
 
 select_fp64 is the same rule on fp64 masses with a plain sequential fp64
 cumulative sum compared against p * total; it serves invariant checks, not
@@ -73,9 +74,9 @@ def _weights(x32: np.ndarray):
 
 
 def select_contract(scores, p: float, scope: str = "row"):
-    """Fixed-point selection on fp32 scores [B, H, nB, nB] -> CSR (row_ptr, col).
+    """Fixed-point selection on fp32 scores [B, H, nQ, nB] -> CSR (row_ptr, col).
 
-    Rows of the CSR are r = (b*H + h)*nB + i; col holds key-block ids.
+    Rows of the CSR are r = (b*H + h)*nQ + i; col holds key-block ids.
     """
     x = np.ascontiguousarray(np.asarray(scores, dtype=np.float32))
     B, H, nQ, nK = x.shape
