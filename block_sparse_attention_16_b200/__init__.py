@@ -26,14 +26,15 @@ __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
     "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule", "lbsa_score_attend",
-    "lbsa_select_head_noalloc", "lbsa_last_error", "lbsa_version", "library_path", "load_library",
+    "lbsa_select_head_noalloc", "lbsa_select_tokens", "lbsa_blockset_views", "lbsa_blockset_masks",
+    "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
 ]
 
 LBSA_OK, LBSA_ERR_INVALID_ARG, LBSA_ERR_UNSUPPORTED, LBSA_ERR_CUDA = 0, 1, 2, 3
 LBSA_ERR_OOM, LBSA_ERR_BAD_INDEX, LBSA_ERR_INVALID_SCORES, LBSA_ERR_TIMEOUT = 4, 5, 6, 7
-_MODES = {"exact": 0, "meanpool": 1}
+_MODES = {"exact": 0, "meanpool": 1, "meanpool_token": 2}
 _SCOPES = {"row": 0, "head": 1}
 _PARTS = {"raster": 0, "1d": 1, "2d": 2, "3d": 3}
 
@@ -78,6 +79,8 @@ def load_library():
         "lbsa_free": (None, [P]),
         "lbsa_blockset_info": (ctypes.c_int, [P] + [ctypes.POINTER(I32)] * 5),
         "lbsa_blockset_views": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P)]),
+        "lbsa_blockset_masks": (ctypes.c_int, [P, ctypes.POINTER(P)]),
+        "lbsa_select_tokens": (ctypes.c_int, [P, I32, I32, I32, I32, D, ctypes.POINTER(P), P]),
         "lbsa_blockset_export": (ctypes.c_int, [P, P, P, ctypes.POINTER(I64), P]),
         "lbsa_blockset_from_csr": (ctypes.c_int, [P, P, I32, I32, I32, I32, ctypes.POINTER(P), P]),
         "lbsa_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32, P]),
@@ -158,13 +161,14 @@ class Blockset:
 
 
 def lbsa_score(q, k, block: int, mode: str = "exact", scores=None, lse=None, want_lse=False, stream=None):
-    """Block scores [B, H, nB, nB] fp32 (and the dense row lse when asked, exact mode)."""
+    """Block scores [B, H, nB, nB] fp32 (and the dense row lse when asked, exact mode);
+    mode "meanpool_token" scores every query token: [B, H, N, nB]."""
     _same_layout(q, k)
     desc = _desc(q)
     B, H, N, _ = q.shape
     nB = -(-N // block)
     if scores is None:
-        scores = torch.empty(B, H, nB, nB, dtype=torch.float32, device=q.device)
+        scores = torch.empty(B, H, N if mode == "meanpool_token" else nB, nB, dtype=torch.float32, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
     _check(load_library().lbsa_score(_ptr(q), _ptr(k), ctypes.byref(desc), block, _MODES[mode],
@@ -183,6 +187,50 @@ def lbsa_select(scores, block: int, p: float = 0.99, scope: str = "row", stream=
     _check(load_library().lbsa_select(_ptr(scores), B, H, nB, block, float(p), _SCOPES[scope],
                                       ctypes.byref(h), _stream(stream)))
     return Blockset(h.value)
+
+
+def lbsa_select_tokens(scores, block: int = 64, p: float = 0.25, stream=None) -> Blockset:
+    """Head-scope selection over the (query token, key block) pairs of fp32
+    scores [B, H, N, nB] into a new per-token blockset (64-token blocks)."""
+    if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, N, nB] tensor")
+    B, H, N, nB = scores.shape
+    if nB != -(-N // block):
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"scores have {nB} key blocks, {N} tokens need {-(-N // block)}")
+    h = ctypes.c_void_p()
+    _check(load_library().lbsa_select_tokens(_ptr(scores), B, H, N, block, float(p), ctypes.byref(h),
+                                             _stream(stream)))
+    return Blockset(h.value)
+
+
+class _DeviceArray:
+    """A device buffer of the library seen through __cuda_array_interface__."""
+
+    def __init__(self, ptr: int, n: int, typestr: str):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (ptr, False), "version": 3}
+
+
+def lbsa_blockset_views(bs: Blockset):
+    """Copies of the blockset's storage: counts [R] int32 and cols [R, nB] int32
+    (row r's first counts[r] entries are its ascending key-block ids)."""
+    c, k = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(load_library().lbsa_blockset_views(bs.handle, ctypes.byref(c), ctypes.byref(k)))
+    R = bs.B * bs.H * bs.nB
+    counts = torch.as_tensor(_DeviceArray(c.value, R, "<i4"), device="cuda").clone()
+    cols = torch.as_tensor(_DeviceArray(k.value, R * bs.nB, "<i4"), device="cuda").clone().view(R, bs.nB)
+    return counts, cols
+
+
+def lbsa_blockset_masks(bs: Blockset):
+    """Copy of a per-token blockset's token sets, int64 [R, nB] (bit u of
+    masks[r, t]: token u of row r's query block keeps its t-th listed key
+    block), or None for blocksets of the other scopes."""
+    m = ctypes.c_void_p()
+    _check(load_library().lbsa_blockset_masks(bs.handle, ctypes.byref(m)))
+    if not m.value:
+        return None
+    R = bs.B * bs.H * bs.nB
+    return torch.as_tensor(_DeviceArray(m.value, R * bs.nB, "<i8"), device="cuda").clone().view(R, bs.nB)
 
 
 def lbsa_score_attend(q, k, v, block: int, scores=None, out=None, lse=None, want_lse=False, stream=None):

@@ -25,6 +25,11 @@
 //              N=d, K=64, P read from TMEM) into TMEM.
 // TMEM columns: [0,64) S0/P0, [64,128) S1/P1, [128,128+d) O.  About 100 KB of
 // shared memory per CTA, so two CTAs (two softmax warpgroups) share an SM.
+//
+// Per-token lists (MASKED, 64-token blocks; VMoBA's per-token selection): an
+// entry of a query block's list also carries the 64-bit set of its tokens that
+// keep the key block; the tile keeps both blocks' sets per key block in shared
+// memory, and a row outside the set gives that block zero probability.
 #include "lbsa_device.cuh"
 
 namespace lbsa {
@@ -50,7 +55,11 @@ struct Layout {
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort, n_entries, pad
   static constexpr int OFF_BITMAP = OFF_MISC + 16;
   static constexpr int OFF_SCHED = OFF_BITMAP + 2 * kMaxWords * 4;
-  static size_t bytes(int nB) { return OFF_SCHED + static_cast<size_t>(nB) * 4 + 1024; }
+  // per-token mask tables (MASKED): two uint64 per key block after the schedule
+  __host__ __device__ static size_t mask_off(int nB) { return (OFF_SCHED + static_cast<size_t>(nB) * 4 + 7) & ~size_t(7); }
+  static size_t bytes(int nB, bool masked = false) {
+    return (masked ? mask_off(nB) + static_cast<size_t>(nB) * 16 : OFF_SCHED + static_cast<size_t>(nB) * 4) + 1024;
+  }
 };
 
 struct Bars {
@@ -80,7 +89,7 @@ __device__ __forceinline__ Bars make_bars(uint8_t* base) {
   return r;
 }
 
-template <int D, bool FUSED>
+template <int D, bool FUSED, bool MASKED>
 __global__ void __launch_bounds__(kThreads, 2)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const AttendArgs args, float scale_log2) {
@@ -105,6 +114,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   uint32_t* bm0 = reinterpret_cast<uint32_t*>(smem + L::OFF_BITMAP);
   uint32_t* bm1 = bm0 + kMaxWords;
   uint32_t* sched = reinterpret_cast<uint32_t*>(smem + L::OFF_SCHED);
+  uint64_t* maskA = reinterpret_cast<uint64_t*>(smem + L::mask_off(nB));   // MASKED: rows 0-63 of the tile
+  uint64_t* maskB = maskA + nB;                                            // MASKED: rows 64-127
   const int nwords = (nB + 31) >> 5;
   // a CTA of this launch already gave up on a wait: skip the work, the call has failed
   if (*reinterpret_cast<volatile int32_t*>(args.status) == LBSA_ERR_TIMEOUT) return;
@@ -135,6 +146,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     bm0[i] = 0;
     bm1[i] = 0;
   }
+  if (MASKED)
+    for (int i = tid; i < 2 * nB; i += kThreads) maskA[i] = 0ull;
   __syncthreads();
   if (warp == 4 && lane == 0) {
     // the Q tile does not depend on the schedule: its load overlaps the build
@@ -179,7 +192,10 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     for (int i = tid; i < c0; i += kThreads) {
       const int c = l0[i];
       if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
-      else atomicOr(&bm0[c >> 5], 1u << (c & 31));
+      else {
+        atomicOr(&bm0[c >> 5], 1u << (c & 31));
+        if (MASKED) maskA[c] = args.masks[row0 * nB + i];
+      }
     }
     if (qb1 >= 0) {
       const long long row1 = row0 + 1;
@@ -188,7 +204,10 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       for (int i = tid; i < c1; i += kThreads) {
         const int c = l1[i];
         if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
-        else atomicOr(&bm1[c >> 5], 1u << (c & 31));
+        else {
+          atomicOr(&bm1[c >> 5], 1u << (c & 31));
+          if (MASKED) maskB[c] = args.masks[row1 * nB + i];
+        }
       }
     }
   }
@@ -345,6 +364,9 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       // warp-uniform: rows 0-63 (warps 0,1) and 64-127 (warps 2,3) are the two halves
       const bool take = (((e >> 30) >> half) & 1u) && nvk > 0;
       const bool full = take && nvk >= 64;
+      // per-token lists: this row's own bit for the key block (not warp-uniform)
+      bool mine = true;
+      if (MASKED) mine = ((half ? maskB : maskA)[e & 0xFFFFu] >> (row & 63)) & 1ull;
       uint32_t r[64];
       tmem_ld32(t_lane + sb * BK, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(t_lane + sb * BK + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -360,7 +382,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         for (int c = 0; c < 64; ++c)
           if (c < nvk) mx4[c & 3] = fmaxf(mx4[c & 3], __uint_as_float(r[c]));
       }
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
+      const float mx = (MASKED && !mine) ? -INFINITY : fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
       const float m_new = fmaxf(m, mx);
       const bool need = (m != -INFINITY) && (m_new > m + 8.0f);
       if (m == -INFINITY) m = m_new;
@@ -417,7 +439,13 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       float sum8[8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) u64_as_f2(sum4[i], sum8[2 * i], sum8[2 * i + 1]);
-      const float bsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      float bsum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      if (MASKED && !mine) {
+        // outside this row's own list: zero probability (values computed above are discarded)
+        bsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
       l += bsum;
       if (FUSED && strip && s < n_chunks) strip[static_cast<long long>(s) * BM + row] = m + __log2f(bsum);   // chunk s's log-sum-exp
       if (s >= 2 && !mbar_wait(bars.o_done + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) {
@@ -529,20 +557,19 @@ cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, con
   dim3 grid(tiles, a.H, a.B);
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
   if (a.nB > kMaxBlocks) return cudaErrorInvalidValue;
-  if (a.d == 128) {
-    const size_t smem = Layout<128>::bytes(a.nB);
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  if (a.masks && a.block != 64) return cudaErrorInvalidValue;
+  const bool masked = a.masks != nullptr;
+  auto go = [&](auto kern, size_t smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attend_bf16_kernel<128, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
-  } else {
-    const size_t smem = Layout<64>::bytes(a.nB);
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attend_bf16_kernel<64, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
-  }
-  return cudaGetLastError();
+    kern<<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
+    return cudaGetLastError();
+  };
+  if (a.d == 128)
+    return masked ? go(attend_bf16_kernel<128, false, true>, Layout<128>::bytes(a.nB, true))
+                  : go(attend_bf16_kernel<128, false, false>, Layout<128>::bytes(a.nB));
+  return masked ? go(attend_bf16_kernel<64, false, true>, Layout<64>::bytes(a.nB, true))
+                : go(attend_bf16_kernel<64, false, false>, Layout<64>::bytes(a.nB));
 }
 
 int g_fused_sms = 0;
@@ -575,16 +602,16 @@ cudaError_t launch_score_attend_bf16(const CUtensorMap* tq, const CUtensorMap* t
   auto smem_of = [](size_t b) { return b < 80 * 1024 ? static_cast<size_t>(80 * 1024) : b; };
   if (a.d == 128) {
     const size_t smem = smem_of(Layout<128>::bytes(a.nB));
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<128, true, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attend_bf16_kernel<128, true><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
+    attend_bf16_kernel<128, true, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
   } else {
     const size_t smem = smem_of(Layout<64>::bytes(a.nB));
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<64, true, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attend_bf16_kernel<64, true><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
+    attend_bf16_kernel<64, true, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
   }
   return cudaGetLastError();
 }

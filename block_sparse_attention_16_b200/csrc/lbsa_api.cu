@@ -150,9 +150,10 @@ long long wait_limit() { return lbsa::kDefaultWaitLimit; }
 
 int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStream_t s, lbsa_blockset** out) {
   const size_t R = static_cast<size_t>(B) * H * nB;
-  const size_t cols_bytes = R * nB * sizeof(int32_t);
+  const size_t cols_bytes = ((R * nB * sizeof(int32_t)) + 255) & ~size_t(255);
   const size_t counts_bytes = ((R * sizeof(int32_t)) + 255) & ~size_t(255);
-  const size_t bytes = counts_bytes + cols_bytes + 256;
+  const size_t mask_bytes = (scope == LBSA_SCOPE_TOKEN) ? R * nB * sizeof(uint64_t) : 0;   // per-token scope only
+  const size_t bytes = counts_bytes + cols_bytes + 256 + mask_bytes;
   void* base = nullptr;
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
@@ -170,6 +171,8 @@ int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStrea
   bs->counts = static_cast<int32_t*>(base);
   bs->cols = reinterpret_cast<int32_t*>(static_cast<char*>(base) + counts_bytes);
   bs->status = reinterpret_cast<int32_t*>(static_cast<char*>(base) + counts_bytes + cols_bytes);
+  bs->masks = mask_bytes ? reinterpret_cast<uint64_t*>(static_cast<char*>(base) + counts_bytes + cols_bytes + 256)
+                         : nullptr;
   bs->stream = s;
   cudaGetDevice(&bs->device);
   e = cudaMemsetAsync(bs->status, 0, sizeof(int32_t), s);
@@ -198,7 +201,8 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
   if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
   if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
   if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
-  if (mode != LBSA_SCORE_EXACT_MASS && mode != LBSA_SCORE_MEANPOOL) return fail(LBSA_ERR_INVALID_ARG, "mode %d", mode);
+  if (mode != LBSA_SCORE_EXACT_MASS && mode != LBSA_SCORE_MEANPOOL && mode != LBSA_SCORE_MEANPOOL_TOKEN)
+    return fail(LBSA_ERR_INVALID_ARG, "mode %d", mode);
   if (lse && mode != LBSA_SCORE_EXACT_MASS) return fail(LBSA_ERR_INVALID_ARG, "lse is only produced in exact mode");
   const int nB = n_blocks(desc->N_valid, block);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -222,9 +226,11 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
       e = lbsa::launch_score_exact_f32(static_cast<const float*>(q), static_cast<const float*>(k), *desc, a, s);
     }
   } else {
-    if ((rc = scratch_alloc(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d), s, &ws)) != LBSA_OK)
+    const bool tokens = mode == LBSA_SCORE_MEANPOOL_TOKEN;
+    const int nQ = tokens ? desc->N_valid : nB;
+    if ((rc = scratch_alloc(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d, nQ), s, &ws)) != LBSA_OK)
       return rc;
-    e = lbsa::launch_meanpool(q, k, *desc, block, nB, scores, ws.ptr, s);
+    e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s);
   }
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_score launch");
   return LBSA_OK;
@@ -348,6 +354,38 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
   return LBSA_OK;
 }
 
+int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_valid, int32_t block, double p,
+                       lbsa_blockset** out, void* stream) {
+  int rc;
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if (B < 1 || H < 1 || n_valid < 1) return fail(LBSA_ERR_INVALID_ARG, "B, H, n_valid must be >= 1");
+  if (block != 64) return fail(LBSA_ERR_UNSUPPORTED, "per-token scope is built for 64-token blocks (block %d)", block);
+  if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
+  const int nB = n_blocks(n_valid, block);
+  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "per-token scope is built for nB <= 1024 (nB %d)", nB);
+  if (static_cast<long long>(n_valid) * nB > 65535ll * 4096)
+    return fail(LBSA_ERR_UNSUPPORTED, "%d tokens x %d blocks per head exceed the histogram grid", n_valid, nB);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  if ((rc = new_blockset(B, H, nB, block, LBSA_SCOPE_TOKEN, p, s, &bs)) != LBSA_OK) return rc;
+  DeviceState* ds = nullptr;
+  Scratch ws;
+  if ((rc = device_state(&ds)) != LBSA_OK ||
+      (rc = scratch_alloc(ds, lbsa::select_head_workspace_bytes(B, H, nB, n_valid), s, &ws)) != LBSA_OK) {
+    lbsa_free(bs);
+    return rc;
+  }
+  cudaError_t e = lbsa::launch_select_tokens(scores, B, H, n_valid, nB, p, bs, ws.ptr, s);
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_select_tokens launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
 int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, const lbsa_blockset* bs,
                 void* out, float* lse, void* stream) {
   int rc;
@@ -366,6 +404,7 @@ int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   lbsa::AttendArgs a{desc->B, desc->H, desc->N_valid, desc->d, bs->block, bs->nB, bs->counts, bs->cols, bs->status,
                      out, desc->stride_b, desc->stride_h, desc->stride_n, lse, wait_limit()};
+  a.masks = bs->masks;
   cudaError_t e;
   if (desc->dtype == LBSA_BF16) {
     CUtensorMap tq, tk, tv;
@@ -394,6 +433,12 @@ int lbsa_blockset_info(const lbsa_blockset* bs, int32_t* B, int32_t* H, int32_t*
   if (nB) *nB = bs->nB;
   if (block) *block = bs->block;
   if (scope) *scope = bs->scope;
+  return LBSA_OK;
+}
+
+int lbsa_blockset_masks(const lbsa_blockset* bs, const uint64_t** masks) {
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (masks) *masks = bs->masks;
   return LBSA_OK;
 }
 

@@ -14,6 +14,7 @@ struct lbsa_blockset {
   double p;
   int32_t* counts;      // device [R]
   int32_t* cols;        // device [R * nB]
+  uint64_t* masks;      // device [R * nB] or NULL: per-token scope, bit t = token t of the query block keeps the entry
   int32_t* status;      // device [1]
   void* base;           // single stream-ordered allocation holding the three arrays
   cudaStream_t stream;  // stream it was created on (freed on it)
@@ -38,6 +39,9 @@ struct AttendArgs {
   float* fscratch;        // n_slots * (128 + 4) * n_chunks floats: per-CTA strips and partials
   int32_t* slots;         // n_slots flags, zero at launch
   int n_slots;
+  // per-token scope (64-token blocks): masks[row * nB + t] is the 64-bit set of
+  // the query block's tokens that keep its t-th listed key block; NULL otherwise
+  const uint64_t* masks = nullptr;
 };
 
 struct ScoreArgs {
@@ -69,8 +73,9 @@ cudaError_t launch_score_exact_f32(const float* q, const float* k, const lbsa_qk
                                    const ScoreArgs& a, cudaStream_t s);
 
 // block-mean proxy (meanpool.cu); workspace holds 2*B*H*nB*d floats + partials
-size_t meanpool_workspace_bytes(int B, int H, int nB, int d);
-cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB,
+// nQ: rows of the score matrix, nB (query-block means) or n_valid (query tokens)
+size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ);
+cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
                             float* scores, void* workspace, cudaStream_t s);
 
 // selection (select.cu)
@@ -80,9 +85,14 @@ cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int
                                lbsa_blockset* bs, cudaStream_t s);
 cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, int n_valid, int32_t* head_floor,
                               cudaStream_t s);
-size_t select_head_workspace_bytes(int B, int H, int nB);
+// nQ: rows of each head's pairs (nB query blocks, or n_valid query tokens); 0 means nB
+size_t select_head_workspace_bytes(int B, int H, int nB, int nQ = 0);
 cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs,
                                void* workspace, cudaStream_t s);
+// per-token scope: nQ = n_valid token rows of nB key blocks, 64-token blocks; writes
+// bs->counts / cols / masks per query block
+cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int nB, double p, lbsa_blockset* bs,
+                                 void* workspace, cudaStream_t s);
 cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col,
                               int32_t* nnz_dev, cudaStream_t s);
 cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blockset* bs,

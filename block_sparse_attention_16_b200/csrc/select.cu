@@ -295,13 +295,14 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
   find_digit(pass, Pfix, keep_all, gh, s, status);
 }
 
-// Ties (bits == tb) per query-block row.  One warp per row.
-__global__ void head_tiecount_kernel(const float* __restrict__ scores, int G, int nB, const HeadState* __restrict__ st,
-                                     int32_t* __restrict__ tiecnt) {
+// Ties (bits == tb) per row of a head's nQ x nB pairs (rows: query blocks, or
+// query tokens in per-token scope).  One warp per row.
+__global__ void head_tiecount_kernel(const float* __restrict__ scores, int G, int nQ, int nB,
+                                     const HeadState* __restrict__ st, int32_t* __restrict__ tiecnt) {
   const int lane = threadIdx.x & 31;
   const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (row >= static_cast<long long>(G) * nB) return;
-  const HeadState* s = st + row / nB;
+  if (row >= static_cast<long long>(G) * nQ) return;
+  const HeadState* s = st + row / nQ;
   if (s->keep_all) return;
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
   int c = 0;
@@ -311,18 +312,18 @@ __global__ void head_tiecount_kernel(const float* __restrict__ scores, int G, in
   if (lane == 0) tiecnt[row] = c;
 }
 
-// Exclusive scan of tie counts within each segment.  grid G, 1024 threads.
-__global__ void head_tiescan_kernel(int nB, const HeadState* __restrict__ st, int32_t* __restrict__ tiecnt) {
+// Exclusive scan of the nQ rows' tie counts within each head.  grid G, 1024 threads.
+__global__ void head_tiescan_kernel(int nQ, const HeadState* __restrict__ st, int32_t* __restrict__ tiecnt) {
   __shared__ int buf[1024];
   __shared__ int carry;
   const int g = blockIdx.x;
   if (st[g].keep_all) return;
-  int32_t* c = tiecnt + static_cast<long long>(g) * nB;
+  int32_t* c = tiecnt + static_cast<long long>(g) * nQ;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
-  for (int base = 0; base < nB; base += 1024) {
+  for (int base = 0; base < nQ; base += 1024) {
     const int i = base + threadIdx.x;
-    const int v = (i < nB) ? c[i] : 0;
+    const int v = (i < nQ) ? c[i] : 0;
     buf[threadIdx.x] = v;
     __syncthreads();
     for (int o = 1; o < 1024; o <<= 1) {
@@ -331,7 +332,7 @@ __global__ void head_tiescan_kernel(int nB, const HeadState* __restrict__ st, in
       buf[threadIdx.x] += add;
       __syncthreads();
     }
-    if (i < nB) c[i] = carry + buf[threadIdx.x] - v;
+    if (i < nQ) c[i] = carry + buf[threadIdx.x] - v;
     __syncthreads();
     if (threadIdx.x == 1023) carry += buf[1023];
     __syncthreads();
@@ -370,6 +371,86 @@ __global__ void head_emit_kernel(const float* __restrict__ scores, int G, int nB
     ties_before += __popc(tmask);
   }
   if (lane == 0) counts[row] = base;
+}
+
+// Per-token scope: emit, for each query block, the key blocks kept by at
+// least one of its (up to 64) tokens, ascending, each with the 64-bit mask of
+// the tokens that keep it.  One CTA (256 threads) per (head, query block):
+// every warp decides 8 token rows in flat order (ties ranked across the head
+// by the scanned per-row tie counts), the keep bits are transposed in shared
+// memory, then the non-empty entries are compacted in ascending order.
+constexpr int kTokMaxB = 1024;                // nB bound of per-token scope
+__global__ void __launch_bounds__(256) token_emit_kernel(const float* __restrict__ scores, int G, int nQ, int nB,
+                                                         const HeadState* __restrict__ st,
+                                                         const int32_t* __restrict__ tiebase,
+                                                         int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+                                                         uint64_t* __restrict__ masks) {
+  __shared__ uint32_t keep[64][kTokMaxB / 32];   // [token][word of key blocks]
+  __shared__ int wsum[8];
+  const int nQB = (nQ + 63) >> 6;
+  const int qb = blockIdx.x % nQB, g = blockIdx.x / nQB;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const HeadState* s = st + g;
+  const int nW = (nB + 31) >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const bool all = s->keep_all;
+  const uint32_t tb = s->tb, need = s->need;
+  for (int tt = warp; tt < 64; tt += 8) {
+    const int r = qb * 64 + tt;
+    if (r >= nQ) {
+      for (int w = lane; w < nW; w += 32) keep[tt][w] = 0u;
+      continue;
+    }
+    const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + (static_cast<long long>(g) * nQ + r) * nB;
+    uint32_t ties_before = all ? 0u : static_cast<uint32_t>(tiebase[static_cast<long long>(g) * nQ + r]);
+    for (int j0 = 0; j0 < nB; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t b = (j < nB) ? __ldg(x + j) : 0u;
+      const bool tie = (j < nB) && b == tb;
+      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+      const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+      const bool k = (j < nB) && (all || b > tb || (tie && rank < need));
+      const uint32_t kmask = __ballot_sync(0xffffffffu, k);
+      if (lane == 0) keep[tt][j0 >> 5] = kmask;
+      ties_before += __popc(tmask);
+    }
+  }
+  __syncthreads();
+  // thread t owns key blocks [t*per, t*per + per): masks, then an ordered compaction
+  const int per = (nB + 255) / 256;
+  const int j_lo = threadIdx.x * per, j_hi = min(nB, j_lo + per);
+  uint64_t m[(kTokMaxB + 255) / 256];
+  int cnt = 0;
+#pragma unroll
+  for (int u = 0; u < (kTokMaxB + 255) / 256; ++u) {
+    m[u] = 0ull;
+    const int j = j_lo + u;
+    if (u < per && j < j_hi) {
+      for (int tt = 0; tt < 64; ++tt) m[u] |= static_cast<uint64_t>((keep[tt][j >> 5] >> (j & 31)) & 1u) << tt;
+      cnt += (m[u] != 0ull);
+    }
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  int pos = incl - cnt;
+  for (int w = 0; w < warp; ++w) pos += wsum[w];
+  const long long row = static_cast<long long>(g) * nQB + qb;
+#pragma unroll
+  for (int u = 0; u < (kTokMaxB + 255) / 256; ++u) {
+    const int j = j_lo + u;
+    if (u < per && j < j_hi && m[u]) {
+      cols[row * nB + pos] = j;
+      masks[row * nB + pos] = m[u];
+      ++pos;
+    }
+  }
+  if (threadIdx.x == 255) counts[row] = pos;
 }
 
 // ---------------------------------------------------------------- CSR export / import
@@ -610,9 +691,10 @@ cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, i
   return cudaGetLastError();
 }
 
-size_t select_head_workspace_bytes(int B, int H, int nB) {
+size_t select_head_workspace_bytes(int B, int H, int nB, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
-  return G * kBins * sizeof(unsigned long long) + G * sizeof(HeadState) + G * nB * sizeof(int32_t) + 256;
+  if (nQ <= 0) nQ = nB;
+  return G * kBins * sizeof(unsigned long long) + G * sizeof(HeadState) + G * nQ * sizeof(int32_t) + 256;
 }
 
 cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs, void* ws,
@@ -633,9 +715,39 @@ cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double
   }
   const long long rows = static_cast<long long>(G) * nB;
   const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie);
+  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, nB, st, tie);
   head_tiescan_kernel<<<G, 1024, 0, s>>>(nB, st, tie);
   head_emit_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie, bs->counts, bs->cols);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int nB, double p, lbsa_blockset* bs,
+                                 void* ws, cudaStream_t s) {
+  if (nB > kTokMaxB) return cudaErrorInvalidValue;
+  const int G = B * H;
+  const long long seg = static_cast<long long>(nQ) * nB;
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(ws);
+  HeadState* st = reinterpret_cast<HeadState*>(hist + static_cast<size_t>(G) * kBins);
+  int32_t* tie = reinterpret_cast<int32_t*>(st + G);
+  cudaError_t e = cudaMemsetAsync(ws, 0, static_cast<size_t>(G) * kBins * sizeof(unsigned long long) +
+                                             static_cast<size_t>(G) * sizeof(HeadState), s);
+  if (e != cudaSuccess) return e;
+  const uint32_t P = fixed_p(p);
+  const int keep_all = p >= 1.0 ? 1 : 0;
+  // one histogram CTA per kHistPerCta pairs (its 32-bit shared sums rely on that bound)
+  const long long chunks = (seg + kHistPerCta - 1) / kHistPerCta;
+  if (chunks > 65535) return cudaErrorInvalidValue;
+  const unsigned hc = static_cast<unsigned>(chunks);
+  for (int pass = 0; pass < 3; ++pass) {
+    head_hist_kernel<<<dim3(hc, G), 256, 0, s>>>(scores, seg, pass, P, keep_all, hist, st, bs->status);
+  }
+  const long long rows = static_cast<long long>(G) * nQ;
+  const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
+  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nQ, nB, st, tie);
+  head_tiescan_kernel<<<G, 1024, 0, s>>>(nQ, st, tie);
+  const int nQB = (nQ + 63) / 64;
+  token_emit_kernel<<<static_cast<unsigned>(G) * nQB, 256, 0, s>>>(scores, G, nQ, nB, st, tie, bs->counts, bs->cols,
+                                                                  bs->masks);
   return cudaGetLastError();
 }
 
@@ -735,7 +847,7 @@ extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t 
   }
   const long long rows = static_cast<long long>(G) * nB;
   const unsigned wblocks = static_cast<unsigned>((rows * 32 + 255) / 256);
-  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie);
+  head_tiecount_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, nB, st, tie);
   head_tiescan_kernel<<<G, 1024, 0, s>>>(nB, st, tie);
   head_emit_kernel<<<wblocks, 256, 0, s>>>(scores, G, nB, st, tie, counts, cols);
   e = cudaGetLastError();

@@ -97,6 +97,8 @@ __global__ void attend_f32_kernel(const float* __restrict__ q, const float* __re
         if (lane == 0) raise_status(a.status, LBSA_ERR_BAD_INDEX);
         continue;
       }
+      // per-token lists (64-token blocks): skip entries this token does not keep
+      if (a.masks && !((a.masks[row * nB + t] >> (r - r0)) & 1ull)) continue;
       const int c1 = min((j + 1) * blk, N);
       for (int c = j * blk; c < c1; ++c) {
         const float s = warp_dot<D>(qr, kh + c * desc.stride_n, lane) * scale;

@@ -62,8 +62,8 @@ typedef enum {
 } lbsa_status;
 
 typedef enum { LBSA_BF16 = 0, LBSA_F32 = 1 } lbsa_dtype;
-typedef enum { LBSA_SCORE_EXACT_MASS = 0, LBSA_SCORE_MEANPOOL = 1 } lbsa_score_mode;
-typedef enum { LBSA_SCOPE_ROW = 0, LBSA_SCOPE_HEAD = 1 } lbsa_scope;
+typedef enum { LBSA_SCORE_EXACT_MASS = 0, LBSA_SCORE_MEANPOOL = 1, LBSA_SCORE_MEANPOOL_TOKEN = 2 } lbsa_score_mode;
+typedef enum { LBSA_SCOPE_ROW = 0, LBSA_SCOPE_HEAD = 1, LBSA_SCOPE_TOKEN = 2 } lbsa_scope;
 typedef enum {
   LBSA_PART_RASTER = 0,         /* identity                                        */
   LBSA_PART_1D = 1,             /* temporal rows: t fastest                        */
@@ -88,7 +88,8 @@ typedef struct lbsa_blockset lbsa_blockset;
 
 /* Stage 1: block scores.
  * LoSA abstract (exact mass) / VMoBA review "What carries the argument"
- * (block-mean proxy).
+ * (block-mean proxy; per-token queries: referee report major comment 1, "full
+ * query-by-block similarity matrix").
  *   q, k    [B, H, N_valid, d] per desc (bf16 or fp32)
  *   block   tokens per block, 64 or 128 (same for queries and keys)
  *   mode    LBSA_SCORE_EXACT_MASS: scores[b,h,i,j] = mean over the valid
@@ -97,7 +98,11 @@ typedef struct lbsa_blockset lbsa_blockset;
  *           LBSA_SCORE_MEANPOOL: qbar_i, kbar_j = means of the valid tokens of
  *           the blocks (fp32), s_ij = qbar_i . kbar_j / sqrt(d),
  *           scores[b,h,:,:] = softmax over all nB*nB pairs of the head.
+ *           LBSA_SCORE_MEANPOOL_TOKEN: every valid query token scores the
+ *           key-block means, s_rj = q_r . kbar_j / sqrt(d), and
+ *           scores[b,h,:,:] = softmax over all N_valid*nB pairs of the head.
  *   scores  out: fp32 [B, H, nB, nB] contiguous, nB = ceil(N_valid / block)
+ *           (LBSA_SCORE_MEANPOOL_TOKEN: [B, H, N_valid, nB])
  *   lse     optional out (exact mode only; NULL to skip): fp32 [B, H, N_valid]
  *           contiguous, natural-log log-sum-exp of each query row of the dense
  *           pass.
@@ -166,6 +171,26 @@ typedef enum { LBSA_RULE_LOCAL_TOPK = 0, LBSA_RULE_TOPP_FLOOR = 1 } lbsa_rule;
 int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, int32_t n_valid,
                      int32_t rule, double p, int32_t k, lbsa_blockset** out, void* stream);
 
+/* Stage 2 at token granularity (VMoBA review: global selection over a head,
+ * here over its (query token, key block) pairs, the pairs of the
+ * LBSA_SCORE_MEANPOOL_TOKEN scores; threshold tau; tokens may keep nothing).
+ *   scores   fp32 [B, H, n_valid, nB] contiguous device array, 0 <= x < 2
+ *   n_valid  valid tokens; nB = ceil(n_valid / 64) <= 1024
+ *   block    must be 64 (a query block's tokens fit one 64-bit mask)
+ *   p        in (0, 1]
+ *   out      receives a new blockset (scope LBSA_SCOPE_TOKEN, free with
+ *            lbsa_free): query block i lists, ascending, every key block that
+ *            at least one of its tokens keeps, each with the 64-bit set of
+ *            those tokens (lbsa_blockset_masks); lbsa_attend then lets token
+ *            r attend to its own kept blocks only.
+ * Rule: as lbsa_select with LBSA_SCOPE_HEAD over the head's n_valid*nB pairs
+ * (flat index r*nB + j, exact fixed-point sums, score descending then flat
+ * index ascending, at least one pair per head).  Invalid scores keep every
+ * pair of the head and set LBSA_ERR_INVALID_SCORES.  Scratch: the radix
+ * histograms and per-token tie counts of B*H heads, from the library pool. */
+int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_valid, int32_t block, double p,
+                       lbsa_blockset** out, void* stream);
+
 /* Stage 3: block-sparse attention over a (frozen) blockset.
  * VMoBA review "What carries the argument" (only selected blocks contribute
  * their key-value pairs); LoSA abstract (frozen indices reused).
@@ -175,7 +200,8 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
  *            same B, H and nB = ceil(N_valid / block)
  *   out      [B, H, N_valid, d], same dtype and strides as q:
  *            out_r = sum_{c in K_i} softmax_{c in K_i}(q_r . k_c / sqrt(d)) v_c
- *            where K_i are the valid keys of the kept blocks of r's block.
+ *            where K_i are the valid keys of the kept blocks of r's block
+ *            (per-token blockset: of the blocks that token r itself keeps).
  *            A row whose list is empty gets 0.
  *   lse      optional fp32 [B, H, N_valid] (natural log; -inf for empty rows).
  * An out-of-range block id in bs is skipped and flags LBSA_ERR_BAD_INDEX in
@@ -194,6 +220,12 @@ int lbsa_blockset_info(const lbsa_blockset* bs, int32_t* B, int32_t* H, int32_t*
  * counts[r] = kept blocks of row r (R = B*H*nB rows); cols[r*nB + t], t <
  * counts[r], ascending key-block ids. */
 int lbsa_blockset_views(const lbsa_blockset* bs, const int32_t** counts, const int32_t** cols);
+
+/* Device view of a per-token blockset's token sets (read-only; valid until
+ * lbsa_free): masks[r*nB + t], t < counts[r], bit u set when token
+ * i*64 + u of query block i keeps the t-th listed key block.  *masks is NULL
+ * for blocksets of the other scopes. */
+int lbsa_blockset_masks(const lbsa_blockset* bs, const uint64_t** masks);
 
 /* Compact CSR export (a helper, not on the per-call path).  row_ptr: device
  * int32 [R + 1]; col: device int32 with room for R*nB entries; *nnz (host)

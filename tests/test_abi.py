@@ -118,3 +118,17 @@ def test_partition_perm_rejects_bad_args():
     assert lib.lbsa_partition_perm(0, 2, 2, 0, 1, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_partition_perm(2, 2, 2, 9, 1, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_partition_perm(2, 2, 2, 3, 0, 1, 1, buf, 0, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+def test_select_tokens_rejects_bad_block_p_and_size():
+    lib = lbsa.load_library()
+    buf = np.zeros(4096, dtype=np.float32)                  # host memory: rejected before any launch
+    h = ctypes.c_void_p()
+    p = ctypes.c_void_p(buf.ctypes.data)
+    assert lib.lbsa_select_tokens(p, 1, 1, 256, 128, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.0, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 1.5, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select_tokens(p, 1, 1, 64 * 1025, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select_tokens(p, 0, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.25, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_select_tokens(None, 1, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
