@@ -59,6 +59,29 @@ def attention_flops(counts, nB, block, n_valid, d):
     return 4.0 * d * float(np.einsum("gij,i,j->", c, valid, valid))
 
 
+def token_flops(lbsa, bs, wl):
+    """Attention FLOPs on the kept (token, key block) pairs of a per-token blockset,
+    4*d*sum over tokens of their kept blocks' valid keys; also the kept-pair
+    density and the fraction of tokens that keep nothing."""
+    counts, cols = (x.cpu().numpy() for x in lbsa.lbsa_blockset_views(bs))
+    masks = lbsa.lbsa_blockset_masks(bs).cpu().numpy().view(np.uint64)
+    nB, blk = wl.n_blocks, wl.block
+    valid = np.full(nB, blk, dtype=np.float64)
+    valid[-1] = wl.n_valid - (nB - 1) * blk
+    slot = np.arange(nB)[None, :] < counts[:, None]
+    m = np.where(slot, masks, np.uint64(0))
+    pop = np.unpackbits(m.view(np.uint8), axis=1).reshape(m.shape[0], nB, 64).sum(-1)     # tokens per entry
+    kept = float(pop.sum())
+    fl = 4.0 * wl.d * float((pop * valid[np.where(slot, cols, 0)]).sum())
+    per_tok = np.zeros((m.shape[0], 64), dtype=np.uint64)
+    for u in range(64):
+        per_tok[:, u] = ((m >> np.uint64(u)) & np.uint64(1)).max(axis=1)
+    G = wl.B * wl.H
+    n_tok = G * wl.n_valid
+    has = per_tok.reshape(G, nB * 64)[:, :wl.n_valid].sum()
+    return fl, kept / (n_tok * nB), 1.0 - float(has) / n_tok
+
+
 def kept_mask(row_ptr, col, rows, nB):
     m = np.zeros((rows, nB), dtype=np.float64)
     r = np.repeat(np.arange(rows), np.diff(row_ptr))
@@ -403,7 +426,8 @@ def load_traffic(kernel):
 def run_profile(kernel):
     """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
     than L2), one warm-up pass of the path, then two launches of `kernel`; or,
-    for "proxy", one mean-pooled proxy call per partition on the full shape."""
+    for "proxy", one mean-pooled proxy call per partition on the full shape; for
+    "token", one call of each per-token proxy stage on the full shape (3D tiles)."""
     import dataclasses
 
     import block_sparse_attention_16_b200 as lbsa
@@ -411,6 +435,20 @@ def run_profile(kernel):
     from block_sparse_attention_16_b200.workload import get_workload, make_qkv
 
     build()
+    if kernel == "token":
+        # per-token proxy path of the Wan-like shape (3D tiles), one call of each stage
+        wl = get_workload("wan_proxy")
+        T, H, W = wl.grid
+        q, k, v = make_qkv(wl, device="cuda")
+        perm = lbsa.lbsa_partition_perm(T, H, W, "3d", device="cuda")
+        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+        sc = lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool_token")
+        bs = lbsa.lbsa_select_tokens(sc, wl.block, 0.25)
+        lbsa.lbsa_attend(qp, kp, vp, bs)
+        torch.cuda.synchronize()
+        assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+        print("profile case token: ok")
+        return 0
     if kernel == "proxy":
         # mean-pooled proxy path of the Wan-like shape, one call per partition
         wl = get_workload("wan_proxy")
@@ -592,6 +630,27 @@ def run_sweep(args):
         emit(workload="wan_proxy", partition=kind, stage="full_call", **tc)
     del q, k, v, qp, kp, vp, sc
 
+    # per-token proxy (VMoBA's literal scoring): every query token scores the key-block
+    # means, head-scope selection at tau = 0.25 over the (token, key block) pairs
+    wl = get_workload("wan_proxy")
+    q, k, v = make_qkv(wl, device="cuda")
+    for kind in ("1d", "2d", "3d"):
+        perm = lbsa.lbsa_partition_perm(T, H, W, kind, device="cuda")
+        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+        sc = lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool_token")
+        bs = lbsa.lbsa_select_tokens(sc, wl.block, 0.25)
+        fl, dens, empty = token_flops(lbsa, bs, wl)
+        tm = _timer(lambda: lbsa.lbsa_score(qp, kp, wl.block, mode="meanpool_token", scores=sc), flush=flush)
+        th = _timer(lambda: lbsa.lbsa_select_tokens(sc, wl.block, 0.25), flush=flush)
+        ta = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+        emit(workload="wan_proxy_token", partition=kind, stage="meanpool_token", **tm,
+             **hbm(2 * q.numel() * 2 + sc.numel() * 4, tm["median"]))
+        emit(workload="wan_proxy_token", partition=kind, stage="select_tokens", **th, **hbm(sc.numel() * 4, th["median"]))
+        emit(workload="wan_proxy_token", partition=kind, stage="attend", density=dens, empty_tokens=empty, **ta,
+             **tfl(fl, ta["median"]))
+        del sc, bs
+    del q, k, v, qp, kp, vp
+
     # HunyuanVideo-like layer: select once, 49 re-drawn attend calls on the frozen blockset
     wl = get_workload("hunyuan")
     q32, k32, v32 = make_qkv_f32(wl, device="cuda")
@@ -632,7 +691,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy"],
+    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy", "token"],
                     help="run the small ncu case for one kernel instead of the benchmark")
     ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
     args = ap.parse_args()
