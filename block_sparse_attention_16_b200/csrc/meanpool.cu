@@ -22,7 +22,6 @@
 namespace lbsa {
 namespace {
 
-constexpr int kTile = 64;
 
 int g_sms = 0;
 int num_sms() {
@@ -158,35 +157,42 @@ __device__ __forceinline__ float4 TokenRows<__nv_bfloat16>::load(int g, int r, i
   return make_float4(a.x, a.y, b.x, b.y);
 }
 
-// grid (nTk, nTq, B*H) with nTk = ceil(nB/64), nTq = ceil(nQ/64); 256 threads,
-// each a 4x4 patch of s.  Rows are the nQ query blocks (qbar, fp32) or, in
-// per-token mode, the nQ = n_valid query tokens read from Q.  Column chunks of
-// the row operand and kbar are staged transposed ([c][row]) so that a thread
-// reads its 4 rows and its 4 columns as one 16-byte load each.
+// grid (nTk, nTq, B*H) with nTk = ceil(nB/128), nTq = ceil(nQ/64); 128 threads.
+// A CTA computes a 64 x 128 tile of s: rows are the nQ query blocks (qbar,
+// fp32) or, in per-token mode, the nQ = n_valid query tokens read from Q;
+// columns are key blocks (kbar).  Thread (y, x) of the 8 x 16 thread grid owns
+// rows {4y..4y+3, 32+4y..32+4y+3} and columns {4x..4x+3, 64+4x..64+4x+3}, so
+// that each 16-byte shared load of a warp (8 x 4 threads) touches distinct
+// bank groups: 4 loads feed 64 FMAs.  Column chunks of 16 of d are staged
+// transposed ([c][row], rows padded by 4) through registers, the next chunk's
+// global loads in flight while the current one is used.  Every s_ij is summed
+// over d in ascending order.
+constexpr int kTq = 64, kTk = 128;
 template <int D, typename TQ, bool TOK>
-__global__ void __launch_bounds__(256) logits_kernel(const TQ* __restrict__ qsrc, long long q_sb, long long q_sh,
+__global__ void __launch_bounds__(128) logits_kernel(const TQ* __restrict__ qsrc, long long q_sb, long long q_sh,
                                                      long long q_sn, int H, const float* __restrict__ kbar, int nQ,
                                                      int nB, float scale, float* __restrict__ scores,
                                                      float2* __restrict__ part) {
-  constexpr int KC = 32;                 // columns of d staged per round
-  constexpr int LD = kTile + 4;          // row stride of the staged chunks (16-byte aligned rows)
-  __shared__ __align__(16) float sq[KC][LD];
-  __shared__ __align__(16) float sk[KC][LD];
-  __shared__ float red_m[8], red_s[8];
+  constexpr int KC = 16;                 // columns of d staged per round
+  constexpr int LQ = kTq + 4, LK = kTk + 4;
+  __shared__ __align__(16) float sq[KC][LQ];
+  __shared__ __align__(16) float sk[KC][LK];
+  __shared__ float red_m[4], red_s[4];
   const int ti = blockIdx.y, tj = blockIdx.x, g = blockIdx.z;
   const int nTk = gridDim.x, nTq = gridDim.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* kb = kbar + static_cast<long long>(g) * nB * D;
-  const int tr = (threadIdx.x / 16) * 4, tc = (threadIdx.x % 16) * 4;
-  float acc[4][4] = {};
-  // the next round's operands are fetched into registers while this round computes
-  float4 na[2], nb[2];
+  const int y = lane >> 2, x = warp * 4 + (lane & 3);
+  float acc[8][8] = {};
+  // staging: the q tile is 64 rows x 4 float4 (2 per thread), the kbar tile
+  // 128 rows x 4 float4 (4 per thread); element e -> row e >> 2, columns 4*(e & 3)
+  float4 na[2], nb[4];
   auto fetch = [&](int c0) {
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
-      const int e = threadIdx.x + it * 256;
-      const int r = e >> 3, c4 = (e & 7) * 4;
-      const int qi = ti * kTile + r, kj = tj * kTile + r;
+      const int e = threadIdx.x + it * 128;
+      const int r = e >> 2, c4 = (e & 3) * 4;
+      const int qi = ti * kTq + r;
       if (qi < nQ) {
         if constexpr (TOK) {
           na[it] = (TokenRows<TQ>{qsrc, q_sb, q_sh, q_sn, H}).load(g, qi, c0 + c4);
@@ -197,70 +203,94 @@ __global__ void __launch_bounds__(256) logits_kernel(const TQ* __restrict__ qsrc
       } else {
         na[it] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+    }
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int e = threadIdx.x + it * 128;
+      const int r = e >> 2, c4 = (e & 3) * 4;
+      const int kj = tj * kTk + r;
       nb[it] = (kj < nB) ? *reinterpret_cast<const float4*>(kb + static_cast<long long>(kj) * D + c0 + c4)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
   fetch(0);
   for (int c0 = 0; c0 < D; c0 += KC) {
-    // 64 rows x 8 float4 per operand: two float4 per thread per operand, stored transposed
 #pragma unroll
     for (int it = 0; it < 2; ++it) {
-      const int e = threadIdx.x + it * 256;
-      const int r = e >> 3, c4 = (e & 7) * 4;
+      const int e = threadIdx.x + it * 128;
+      const int r = e >> 2, c4 = (e & 3) * 4;
       sq[c4][r] = na[it].x; sq[c4 + 1][r] = na[it].y; sq[c4 + 2][r] = na[it].z; sq[c4 + 3][r] = na[it].w;
+    }
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int e = threadIdx.x + it * 128;
+      const int r = e >> 2, c4 = (e & 3) * 4;
       sk[c4][r] = nb[it].x; sk[c4 + 1][r] = nb[it].y; sk[c4 + 2][r] = nb[it].z; sk[c4 + 3][r] = nb[it].w;
     }
     __syncthreads();
     if (c0 + KC < D) fetch(c0 + KC);
-#pragma unroll 8
+#pragma unroll
     for (int c = 0; c < KC; ++c) {
-      const float4 a = *reinterpret_cast<const float4*>(&sq[c][tr]);
-      const float4 b = *reinterpret_cast<const float4*>(&sk[c][tc]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+      const float4 a0 = *reinterpret_cast<const float4*>(&sq[c][4 * y]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sq[c][32 + 4 * y]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&sk[c][4 * x]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sk[c][64 + 4 * x]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
 #pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
     }
     __syncthreads();
   }
+  // epilogue: scale, store (16-byte vectors where the 4 columns are in range), tile (max, sum of exp)
   float mx = -INFINITY;
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int u = 0; u < 8; ++u) {
+    const int qi = ti * kTq + (u < 4 ? 4 * y + u : 32 + 4 * y + u - 4);
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int qi = ti * kTile + tr + u, kj = tj * kTile + tc + w;
-      acc[u][w] *= scale;
-      if (qi < nQ && kj < nB) {
-        scores[(static_cast<long long>(g) * nQ + qi) * nB + kj] = acc[u][w];
-        mx = fmaxf(mx, acc[u][w]);
+    for (int w = 0; w < 8; ++w) acc[u][w] *= scale;
+    if (qi >= nQ) continue;
+#pragma unroll
+    for (int hx = 0; hx < 2; ++hx) {
+      const int kj0 = tj * kTk + hx * 64 + 4 * x;
+      float* dst = scores + (static_cast<long long>(g) * nQ + qi) * nB + kj0;
+      const float* a = &acc[u][4 * hx];
+      if ((nB & 3) == 0 && kj0 + 3 < nB) {
+        *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
+        mx = fmaxf(mx, fmaxf(fmaxf(a[0], a[1]), fmaxf(a[2], a[3])));
+      } else {
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (kj0 + w < nB) {
+            dst[w] = a[w];
+            mx = fmaxf(mx, a[w]);
+          }
       }
     }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (lane == 0) red_m[warp] = mx;
   __syncthreads();
-  float tm = red_m[0];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) tm = fmaxf(tm, red_m[w]);
+  const float tm = fmaxf(fmaxf(red_m[0], red_m[1]), fmaxf(red_m[2], red_m[3]));
   float sm = 0.f;
 #pragma unroll
-  for (int u = 0; u < 4; ++u)
+  for (int u = 0; u < 8; ++u) {
+    const int qi = ti * kTq + (u < 4 ? 4 * y + u : 32 + 4 * y + u - 4);
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int qi = ti * kTile + tr + u, kj = tj * kTile + tc + w;
+    for (int w = 0; w < 8; ++w) {
+      const int kj = tj * kTk + (w < 4 ? 4 * x + w : 64 + 4 * x + w - 4);
       if (qi < nQ && kj < nB) sm += expf(acc[u][w] - tm);
     }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
   if (lane == 0) red_s[warp] = sm;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float z = 0.f;
-    for (int w = 0; w < 8; ++w) z += red_s[w];
-    part[(static_cast<long long>(g) * nTq + ti) * nTk + tj] = make_float2(tm, z);
-  }
+  if (threadIdx.x == 0)
+    part[(static_cast<long long>(g) * nTq + ti) * nTk + tj] = make_float2(tm, (red_s[0] + red_s[1]) + (red_s[2] + red_s[3]));
 }
 
 // grid (chunks, B*H), 256 threads: warp 0 combines the head's tile partials
@@ -372,7 +402,7 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
   float* kbar = qbar + G * nB * D;
   float2* part = reinterpret_cast<float2*>(kbar + G * nB * D);
   const int nQ = tokens ? d.N_valid : nB;
-  const int nTk = (nB + kTile - 1) / kTile, nTq = (nQ + kTile - 1) / kTile;
+  const int nTk = (nB + kTk - 1) / kTk, nTq = (nQ + kTq - 1) / kTq;
   const long long items = G * nB;
   if (d.dtype == LBSA_BF16) {
     if (block <= 64)
@@ -388,13 +418,13 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const dim3 lgrid(nTk, nTq, static_cast<unsigned>(G));
   if (!tokens) {
-    logits_kernel<D, float, false><<<lgrid, 256, 0, s>>>(qbar, 0, 0, 0, d.H, kbar, nQ, nB, scale, scores, part);
+    logits_kernel<D, float, false><<<lgrid, 128, 0, s>>>(qbar, 0, 0, 0, d.H, kbar, nQ, nB, scale, scores, part);
   } else if (d.dtype == LBSA_BF16) {
-    logits_kernel<D, __nv_bfloat16, true><<<lgrid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(q), d.stride_b,
+    logits_kernel<D, __nv_bfloat16, true><<<lgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(q), d.stride_b,
                                                                  d.stride_h, d.stride_n, d.H, kbar, nQ, nB, scale,
                                                                  scores, part);
   } else {
-    logits_kernel<D, float, true><<<lgrid, 256, 0, s>>>(static_cast<const float*>(q), d.stride_b, d.stride_h,
+    logits_kernel<D, float, true><<<lgrid, 128, 0, s>>>(static_cast<const float*>(q), d.stride_b, d.stride_h,
                                                          d.stride_n, d.H, kbar, nQ, nB, scale, scores, part);
   }
   const long long n = static_cast<long long>(nQ) * nB;
@@ -413,7 +443,7 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
 
 size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
-  const size_t nTk = (nB + kTile - 1) / kTile, nTq = (nQ + kTile - 1) / kTile;
+  const size_t nTk = (nB + kTk - 1) / kTk, nTq = (nQ + kTq - 1) / kTq;
   return 2 * G * nB * d * sizeof(float) + (G * nTq * nTk + G) * sizeof(float2) + 256;
 }
 
