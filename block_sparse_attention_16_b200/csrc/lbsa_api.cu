@@ -16,6 +16,25 @@ namespace {
 
 thread_local std::string g_err;
 
+// Host-side call log: with LBSA_LOG set to a non-empty value other than "0",
+// every entry point and every non-OK return writes one line to stderr.
+bool log_on() {
+  static const bool on = [] {
+    const char* v = std::getenv("LBSA_LOG");
+    return v && *v && std::strcmp(v, "0") != 0;
+  }();
+  return on;
+}
+void log_line(const char* fmt, ...) {
+  if (!log_on()) return;
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  std::fprintf(stderr, "[lbsa] %s\n", buf);
+}
+
 int fail(int code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -23,6 +42,7 @@ int fail(int code, const char* fmt, ...) {
   std::vsnprintf(buf, sizeof(buf), fmt, ap);
   va_end(ap);
   g_err = buf;
+  log_line("error %d: %s", code, buf);
   return code;
 }
 
@@ -196,6 +216,9 @@ const char* lbsa_last_error(void) { return g_err.c_str(); }
 int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t block, int32_t mode, float* scores,
                float* lse, void* stream) {
   int rc;
+  if (desc)
+    log_line("lbsa_score mode=%d B=%d H=%d N=%d d=%d dtype=%d block=%d lse=%d", mode, desc->B, desc->H, desc->N_valid,
+             desc->d, desc->dtype, block, lse != nullptr);
   if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
   if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
   if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
@@ -239,6 +262,9 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
 int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, int32_t block,
                       float* scores, void* out, float* lse, void* stream) {
   int rc;
+  if (desc)
+    log_line("lbsa_score_attend B=%d H=%d N=%d d=%d dtype=%d block=%d lse=%d", desc->B, desc->H, desc->N_valid,
+             desc->d, desc->dtype, block, lse != nullptr);
   if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
   if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
   if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
@@ -274,6 +300,7 @@ int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qk
 int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p, int32_t scope,
                 lbsa_blockset** out, void* stream) {
   int rc;
+  log_line("lbsa_select B=%d H=%d nB=%d block=%d p=%.9g scope=%d", B, H, nB, block, p, scope);
   if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
@@ -310,6 +337,8 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
 int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, int32_t n_valid,
                      int32_t rule, double p, int32_t k, lbsa_blockset** out, void* stream) {
   int rc;
+  log_line("lbsa_select_rule B=%d H=%d nB=%d block=%d n_valid=%d rule=%d p=%.9g k=%d", B, H, nB, block, n_valid, rule,
+           p, k);
   if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
@@ -357,6 +386,7 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
 int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_valid, int32_t block, double p,
                        lbsa_blockset** out, void* stream) {
   int rc;
+  log_line("lbsa_select_tokens B=%d H=%d n_valid=%d block=%d p=%.9g", B, H, n_valid, block, p);
   if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
   *out = nullptr;
   if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
@@ -389,6 +419,9 @@ int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_vali
 int lbsa_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, const lbsa_blockset* bs,
                 void* out, float* lse, void* stream) {
   int rc;
+  if (desc)
+    log_line("lbsa_attend B=%d H=%d N=%d d=%d dtype=%d blockset=%p (scope %d) lse=%d", desc->B, desc->H, desc->N_valid,
+             desc->d, desc->dtype, static_cast<const void*>(bs), bs ? bs->scope : -1, lse != nullptr);
   if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
   if ((rc = validate_ptr(q, "q")) != LBSA_OK) return rc;
   if ((rc = validate_ptr(k, "k")) != LBSA_OK) return rc;
@@ -527,6 +560,8 @@ int lbsa_partition_perm(int32_t T, int32_t Hg, int32_t Wg, int32_t kind, int32_t
 int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const int32_t* perm, const lbsa_qkv_desc* desc,
                  int32_t inverse, void* stream) {
   int rc;
+  if (desc) log_line("lbsa_permute count=%d B=%d H=%d N=%d d=%d inverse=%d", count, desc->B, desc->H, desc->N_valid,
+                     desc->d, inverse);
   if ((rc = validate_desc(desc)) != LBSA_OK) return rc;
   if (!xs || !ys || count < 1 || count > 3) return fail(LBSA_ERR_INVALID_ARG, "need 1..3 tensors");
   if (!perm) return fail(LBSA_ERR_INVALID_ARG, "perm is NULL");

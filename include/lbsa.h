@@ -302,7 +302,10 @@ int lbsa_selftest_exp2(const float* v, float* out, int64_t n, void* stream);
 int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t H, int32_t nB, double p,
                              int32_t* counts, int32_t* cols, int32_t* status, void* stream);
 
-/* Thread-local one-line reason for the last non-OK return of this thread. */
+/* Thread-local one-line reason for the last non-OK return of this thread.
+ * With the environment variable LBSA_LOG set (to anything but "" or "0") when
+ * the library first checks it, every entry point and every non-OK return
+ * also writes one line to stderr ("[lbsa] ..."): arguments, shapes, reasons. */
 const char* lbsa_last_error(void);
 
 /* Library ABI version (major * 100 + minor). */

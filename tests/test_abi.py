@@ -132,3 +132,31 @@ def test_select_tokens_rejects_bad_block_p_and_size():
     assert lib.lbsa_select_tokens(p, 0, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.25, None, None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(None, 1, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+def test_call_log_reports_calls_and_errors():
+    """LBSA_LOG=1: the rejected calls of a fresh process each leave a call line and an error line on stderr."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, numpy as np\n"
+        "import block_sparse_attention_16_b200 as lbsa\n"
+        "lib = lbsa.load_library()\n"
+        "buf = np.zeros(64, dtype=np.float32)\n"
+        "h = ctypes.c_void_p()\n"
+        "rc = lib.lbsa_select(ctypes.c_void_p(buf.ctypes.data), 1, 1, 8, 64, 1.5, 0, ctypes.byref(h), None)\n"
+        "rc2 = lib.lbsa_select_tokens(ctypes.c_void_p(buf.ctypes.data), 1, 1, 256, 128, 0.25, ctypes.byref(h), None)\n"
+        "print(rc, rc2)\n")
+    env = dict(os.environ, LBSA_LOG="1")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                       cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == [str(lbsa.LBSA_ERR_INVALID_ARG), str(lbsa.LBSA_ERR_UNSUPPORTED)]
+    lines = [l for l in r.stderr.splitlines() if l.startswith("[lbsa]")]
+    assert any("lbsa_select B=1 H=1 nB=8 block=64 p=1.5" in l for l in lines), lines
+    assert any(l.startswith("[lbsa] error 1:") and "p = 1.5" in l for l in lines), lines
+    assert any("lbsa_select_tokens" in l for l in lines) and any(l.startswith("[lbsa] error 2:") for l in lines), lines
+    quiet = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                           env=dict(os.environ, LBSA_LOG="0"),
+                           cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=120)
+    assert "[lbsa]" not in quiet.stderr
