@@ -254,20 +254,34 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + static_cast<long long>(g) * seg_len;
   unsigned int lmax = 0;
   int lbad = 0;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < seg_len;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const uint32_t b = __ldg(x + i);
-    if (b >= kInvalidBits) {
-      lbad = 1;
-      continue;
+  // a thread's elements (16 at the launch's grid of one CTA per kHistPerCta)
+  // are all loaded before any is binned, so their DRAM round trips overlap
+  constexpr int kBatch = 16;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < seg_len;
+       i0 += kBatch * stride) {
+    uint32_t v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const long long i = i0 + u * stride;
+      v[u] = (i < seg_len) ? __ldg(x + i) : 0u;
     }
-    if (pass == 0) lmax = max(lmax, b);
-    if (pass > 0 && (b >> (shift + kDigitBits)) != prefix) continue;
-    const uint64_t w = fixed_weight(b);
-    if (w) {
-      const uint32_t bin = (b >> shift) & (kBins - 1);
-      atomicAdd(&sh_lo[bin], static_cast<uint32_t>(w & 0xFFFFFull));
-      atomicAdd(&sh_hi[bin], static_cast<uint32_t>(w >> 20));
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (i0 + u * stride >= seg_len) break;
+      const uint32_t b = v[u];
+      if (b >= kInvalidBits) {
+        lbad = 1;
+        continue;
+      }
+      if (pass == 0) lmax = max(lmax, b);
+      if (pass > 0 && (b >> (shift + kDigitBits)) != prefix) continue;
+      const uint64_t w = fixed_weight(b);
+      if (w) {
+        const uint32_t bin = (b >> shift) & (kBins - 1);
+        atomicAdd(&sh_lo[bin], static_cast<uint32_t>(w & 0xFFFFFull));
+        atomicAdd(&sh_hi[bin], static_cast<uint32_t>(w >> 20));
+      }
     }
   }
   if (pass == 0) {
