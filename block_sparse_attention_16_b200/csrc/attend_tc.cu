@@ -186,27 +186,31 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       if (slot < 0) misc[2] = 0;              // no steps: the CTA leaves without work
     }
   } else {
+    // both rows' counts, then both lists, with their loads in flight together
     const long long row0 = (static_cast<long long>(bb) * args.H + h) * nB + qb0;
+    const long long row1 = row0 + 1;
     const int c0 = args.counts[row0];
+    const int c1 = (qb1 >= 0) ? args.counts[row1] : 0;
     const int32_t* l0 = args.cols + row0 * nB;
-    for (int i = tid; i < c0; i += kThreads) {
-      const int c = l0[i];
-      if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
-      else {
-        atomicOr(&bm0[c >> 5], 1u << (c & 31));
-        if (MASKED) maskA[c] = args.masks[row0 * nB + i];
-      }
-    }
-    if (qb1 >= 0) {
-      const long long row1 = row0 + 1;
-      const int c1 = args.counts[row1];
-      const int32_t* l1 = args.cols + row1 * nB;
-      for (int i = tid; i < c1; i += kThreads) {
-        const int c = l1[i];
-        if (c < 0 || c >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
+    const int32_t* l1 = args.cols + row1 * nB;
+    for (int i = tid; i < max(c0, c1); i += kThreads) {
+      const bool h0 = i < c0, h1 = i < c1;
+      const int a = h0 ? l0[i] : 0;
+      const int b = h1 ? l1[i] : 0;
+      const uint64_t ma = (MASKED && h0) ? args.masks[row0 * nB + i] : 0ull;
+      const uint64_t mb = (MASKED && h1) ? args.masks[row1 * nB + i] : 0ull;
+      if (h0) {
+        if (a < 0 || a >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
         else {
-          atomicOr(&bm1[c >> 5], 1u << (c & 31));
-          if (MASKED) maskB[c] = args.masks[row1 * nB + i];
+          atomicOr(&bm0[a >> 5], 1u << (a & 31));
+          if (MASKED) maskA[a] = ma;
+        }
+      }
+      if (h1) {
+        if (b < 0 || b >= nB) raise_status(args.status, LBSA_ERR_BAD_INDEX);
+        else {
+          atomicOr(&bm1[b >> 5], 1u << (b & 31));
+          if (MASKED) maskB[b] = mb;
         }
       }
     }
