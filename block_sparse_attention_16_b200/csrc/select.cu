@@ -35,10 +35,15 @@ __device__ __forceinline__ uint64_t fixed_weight(uint32_t bits) {
   return sh >= 24 ? 0 : (M >> sh);
 }
 
+// Exact warp sum of per-lane values below 2^54: the low 27 bits and the rest
+// are summed separately by two redux.sync adds (each total fits 32 bits),
+// a shorter dependent chain than five rounds of 64-bit shuffles.
 __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+  const uint32_t lo = static_cast<uint32_t>(v) & ((1u << 27) - 1u);
+  const uint32_t hi = static_cast<uint32_t>(v >> 27);
+  const uint32_t slo = __reduce_add_sync(0xffffffffu, lo);
+  const uint32_t shi = __reduce_add_sync(0xffffffffu, hi);
+  return (static_cast<uint64_t>(shi) << 27) + slo;
 }
 
 __device__ __forceinline__ uint64_t threshold_T(uint64_t W, uint32_t Pfix) {
