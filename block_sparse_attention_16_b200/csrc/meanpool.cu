@@ -183,7 +183,12 @@ __global__ void __launch_bounds__(128) logits_kernel(const TQ* __restrict__ qsrc
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* kb = kbar + static_cast<long long>(g) * nB * D;
   const int y = lane >> 2, x = warp * 4 + (lane & 3);
-  float acc[8][8] = {};
+  // accumulators as packed pairs of adjacent columns: acc2[u][v] = (s[u][2v], s[u][2v+1])
+  unsigned long long acc2[8][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc2[u][v] = 0ull;
   // staging: the q tile is 64 rows x 4 float4 (2 per thread), the kbar tile
   // 128 rows x 4 float4 (4 per thread); element e -> row e >> 2, columns 4*(e & 3)
   float4 na[2], nb[4];
@@ -236,15 +241,24 @@ __global__ void __launch_bounds__(128) logits_kernel(const TQ* __restrict__ qsrc
       const float4 b0 = *reinterpret_cast<const float4*>(&sk[c][4 * x]);
       const float4 b1 = *reinterpret_cast<const float4*>(&sk[c][64 + 4 * x]);
       const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const unsigned long long bp[4] = {f2_as_u64(b0.x, b0.y), f2_as_u64(b0.z, b0.w), f2_as_u64(b1.x, b1.y),
+                                        f2_as_u64(b1.z, b1.w)};
+      // packed fp32x2 FMAs (each half an ordinary fp32 FMA: the same sums as scalar FMAs)
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < 8; ++u) {
+        const unsigned long long ap = f2_as_u64(av[u], av[u]);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+        for (int v = 0; v < 4; ++v) acc2[u][v] = ffma2(ap, bp[v], acc2[u][v]);
+      }
     }
     __syncthreads();
   }
   // epilogue: scale, store (16-byte vectors where the 4 columns are in range), tile (max, sum of exp)
+  float acc[8][8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) u64_as_f2(acc2[u][v], acc[u][2 * v], acc[u][2 * v + 1]);
   float mx = -INFINITY;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
