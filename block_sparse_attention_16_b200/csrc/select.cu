@@ -326,8 +326,7 @@ __global__ void head_tiecount_kernel(const float* __restrict__ scores, int G, in
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
   int c = 0;
   for (int j = lane; j < nB; j += 32) c += (__ldg(x + j) == s->tb);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  c = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(c));
   if (lane == 0) tiecnt[row] = c;
 }
 
@@ -594,8 +593,7 @@ __global__ void __launch_bounds__(256) select_rank_kernel(const float* __restric
         const int idx = e * 32 + lane;
         c += (idx < nB && idx != diag && bits[e] >= mid) ? 1u : 0u;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+      c = __reduce_add_sync(0xffffffffu, c);
       if (c >= static_cast<uint32_t>(n)) lo = mid;
       else hi = mid;
     }
@@ -606,8 +604,7 @@ __global__ void __launch_bounds__(256) select_rank_kernel(const float* __restric
       const int idx = e * 32 + lane;
       above += (idx < nB && idx != diag && bits[e] > tb) ? 1u : 0u;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    above = __reduce_add_sync(0xffffffffu, above);
     need = static_cast<uint32_t>(n) - above;
   }
   // emit in ascending id order: the own block (mode 0), the ids ranked above tb,
