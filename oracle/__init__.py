@@ -17,6 +17,9 @@ computes, written from the pages' prose:
     "Local + TopK" selection of the training-free experiments.
   * SCOPE (abstract, mlsift.com): hybrid Top-p with a head-specific Top-k
     floor from the size-weighted mean of the initially retained counts.
+  * EG-Sparse (abstract, readsearch.ai page of arXiv 2610.14672): low-entropy
+    heads routed to a grouped cross-head pool, per-row selection for the
+    high-entropy heads, from the scores already materialised.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It imports nothing from the CUDA library or its
@@ -28,6 +31,8 @@ Modules
   select      select_contract, select_fp64, csr tools  (pinned)
   select_variants  select_local_topk (VMoBA "Local + TopK"), select_topp_floor
               (SCOPE-style per-head floor over row top-p)   (pinned)
+  select_routed  head_entropy, route_heads, select_routed (EG-Sparse
+              entropy-routed competition domains)    (pinned)
   partition   raster / 1D / 2D / 3D token orders       (pinned)
 
 Every function is pinned by a ``-m "not gpu"`` test against something other
@@ -39,6 +44,7 @@ from .scores import block_mass, meanpool_scores, token_meanpool_scores
 from .select import (select_contract, select_fp64, InvalidScores, threshold_fixed_point,
                      csr_rows, csr_from_rows)
 from .select_variants import select_local_topk, select_topp_floor, floor_of_head
+from .select_routed import head_entropy, route_heads, select_routed
 from .partition import (perm_raster, perm_1d_temporal, perm_2d_frame_tiles, perm_3d_tiles,
                         perm_for_call, PARTITION_CYCLE)
 
@@ -47,6 +53,7 @@ __all__ = [
     "token_meanpool_scores",
     "select_contract", "select_fp64", "InvalidScores", "threshold_fixed_point",
     "csr_rows", "csr_from_rows", "select_local_topk", "select_topp_floor", "floor_of_head",
+    "head_entropy", "route_heads", "select_routed",
     "perm_raster", "perm_1d_temporal", "perm_2d_frame_tiles", "perm_3d_tiles",
     "perm_for_call", "PARTITION_CYCLE",
 ]
