@@ -449,6 +449,25 @@ def run_profile(kernel):
         assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
         print("profile case token: ok")
         return 0
+    if kernel == "routed":
+        # entropy-routed selection on the skewed Wan-like layer's exact scores:
+        # heads below the median entropy pooled 3 at a time, p = 0.99; two calls
+        wl = get_workload("wan_skew")
+        T, H, W = wl.grid
+        q, k, v = make_qkv(wl, device="cuda")
+        perm = lbsa.lbsa_partition_perm(T, H, W, "3d", device="cuda")
+        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+        sc = lbsa.lbsa_score(qp, kp, wl.block)
+        _, ent, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, -1.0, 1)
+        e_sorted = ent[0].sort().values
+        thr = float((e_sorted[wl.H // 2 - 1] + e_sorted[wl.H // 2]) / 2)
+        for _ in range(2):
+            bs, _, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, thr, 3)
+        lbsa.lbsa_attend(qp, kp, vp, bs)
+        torch.cuda.synchronize()
+        assert lbsa.lbsa_get_status(bs) == 0 and lbsa.lbsa_device_status() == 0
+        print("profile case routed: ok")
+        return 0
     if kernel == "proxy":
         # mean-pooled proxy path of the Wan-like shape, one call per partition
         wl = get_workload("wan_proxy")
@@ -598,6 +617,22 @@ def run_sweep(args):
         emit(workload="wan_skew", stage="attend", rule=rule, **kw, density=float(m.mean()),
              density_per_head=[round(float(x), 4) for x in m.mean(axis=(1, 2))], **ta, **tfl(fl, ta["median"]),
              select_ms=ts["median"], **{"select_" + k2: v2 for k2, v2 in hbm(sc.numel() * 4, ts["median"]).items()})
+    # entropy-routed competition domains (EG-Sparse): heads below the median
+    # entropy pooled `group` at a time, the rest per row, p = 0.99; and the
+    # all-head pool of the abstract's diagnostic (every head routed, one pool)
+    _, ent, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, -1.0, 1)
+    e_sorted = ent[0].sort().values
+    thr = float((e_sorted[wl.H // 2 - 1] + e_sorted[wl.H // 2]) / 2)
+    for thr_, group in ((thr, 3), (thr, 6), (thr, wl.H), (2.0, wl.H)):
+        bs, _, dom = lbsa.lbsa_select_routed(sc, wl.block, 0.99, thr_, group)
+        fl, m = flops_of(bs, wl)
+        ta = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs))
+        ts = _timer(lambda: lbsa.lbsa_select_routed(sc, wl.block, 0.99, thr_, group), flush=flush)
+        emit(workload="wan_skew", stage="attend", rule="routed", p=0.99, entropy_threshold=round(thr_, 6),
+             group=group, routed_heads=int((dom >= 0).sum()), entropy=[round(float(x), 4) for x in ent[0]],
+             density=float(m.mean()), density_per_head=[round(float(x), 4) for x in m.mean(axis=(1, 2))],
+             empty_rows=float((m.sum(axis=2) == 0).mean()), **ta, **tfl(fl, ta["median"]), select_ms=ts["median"],
+             **{"select_" + k2: v2 for k2, v2 in hbm(sc.numel() * 4, ts["median"]).items()})
     del q, k, v, qp, kp, vp, sc
 
     # proxy mode: 1D / 2D / 3D cycle, head-scope selection at tau = 0.25
@@ -691,7 +726,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy", "token"],
+    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy", "token", "routed"],
                     help="run the small ncu case for one kernel instead of the benchmark")
     ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
     args = ap.parse_args()

@@ -26,7 +26,8 @@ __all__ = [
     "LbsaError", "Blockset", "lbsa_score", "lbsa_select", "lbsa_attend", "lbsa_free",
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
     "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule", "lbsa_score_attend",
-    "lbsa_select_head_noalloc", "lbsa_select_tokens", "lbsa_blockset_views", "lbsa_blockset_masks",
+    "lbsa_select_head_noalloc", "lbsa_select_tokens", "lbsa_select_routed", "lbsa_blockset_views",
+    "lbsa_blockset_masks",
     "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
@@ -81,6 +82,7 @@ def load_library():
         "lbsa_blockset_views": (ctypes.c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P)]),
         "lbsa_blockset_masks": (ctypes.c_int, [P, ctypes.POINTER(P)]),
         "lbsa_select_tokens": (ctypes.c_int, [P, I32, I32, I32, I32, D, ctypes.POINTER(P), P]),
+        "lbsa_select_routed": (ctypes.c_int, [P, I32, I32, I32, I32, D, D, I32, P, P, ctypes.POINTER(P), P]),
         "lbsa_blockset_export": (ctypes.c_int, [P, P, P, ctypes.POINTER(I64), P]),
         "lbsa_blockset_from_csr": (ctypes.c_int, [P, P, I32, I32, I32, I32, ctypes.POINTER(P), P]),
         "lbsa_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32, P]),
@@ -273,6 +275,25 @@ def lbsa_select_rule(scores, block: int, rule: str, n_valid: int, p: float = 0.9
     _check(load_library().lbsa_select_rule(_ptr(scores), B, H, nB, block, int(n_valid), _RULES[rule], float(p),
                                            int(k), ctypes.byref(h), _stream(stream)))
     return Blockset(h.value)
+
+
+def lbsa_select_routed(scores, block: int, p: float, entropy_threshold: float, group: int, stream=None):
+    """Entropy-routed selection into a new blockset: heads whose normalised
+    mean row entropy is below entropy_threshold are pooled, `group` at a time
+    in head order, and each pool's rows of one query block compete together;
+    the other heads take the row rule.  Returns (blockset, head entropy fp64
+    [B, H], head domain int32 [B, H]: -1 per row, else the pool index)."""
+    if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, nB, nB] tensor")
+    B, H, nB, nB2 = scores.shape
+    if nB != nB2:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be square per head")
+    ent = torch.empty(B, H, dtype=torch.float64, device=scores.device)
+    dom = torch.empty(B, H, dtype=torch.int32, device=scores.device)
+    h = ctypes.c_void_p()
+    _check(load_library().lbsa_select_routed(_ptr(scores), B, H, nB, block, float(p), float(entropy_threshold),
+                                             int(group), _ptr(ent), _ptr(dom), ctypes.byref(h), _stream(stream)))
+    return Blockset(h.value), ent, dom
 
 
 def lbsa_attend(q, k, v, bs: Blockset, out=None, lse=None, want_lse=False, stream=None):

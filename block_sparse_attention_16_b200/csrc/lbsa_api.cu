@@ -209,7 +209,7 @@ int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStrea
 
 extern "C" {
 
-int lbsa_version(void) { return 100; }
+int lbsa_version(void) { return 101; }
 
 const char* lbsa_last_error(void) { return g_err.c_str(); }
 
@@ -411,6 +411,48 @@ int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_vali
   if (e != cudaSuccess) {
     lbsa_free(bs);
     return cuda_fail(e, "lbsa_select_tokens launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
+int lbsa_select_routed(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,
+                       double entropy_threshold, int32_t group, double* head_entropy, int32_t* head_domain,
+                       lbsa_blockset** out, void* stream) {
+  int rc;
+  log_line("lbsa_select_routed B=%d H=%d nB=%d block=%d p=%.9g threshold=%.9g group=%d", B, H, nB, block, p,
+           entropy_threshold, group);
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
+  if (B < 1 || H < 1 || nB < 1) return fail(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
+  if (std::isnan(entropy_threshold)) return fail(LBSA_ERR_INVALID_ARG, "entropy threshold is NaN");
+  if (group < 1) return fail(LBSA_ERR_INVALID_ARG, "group = %d < 1", group);
+  if (H > 4096) return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for H <= 4096 (H %d)", H);
+  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for nB <= 1024 (nB %d)", nB);
+  if (static_cast<long long>(B) * H > 65535)
+    return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for B*H <= 65535 heads (%d x %d)", B, H);
+  const size_t smem = lbsa::select_routed_smem_bytes(H, nB, group);
+  if (smem > 200 * 1024)
+    return fail(LBSA_ERR_UNSUPPORTED, "a pool of %d heads x %d key blocks needs %zu bytes of shared memory (> 200 KiB)",
+                group < H ? group : H, nB, smem);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  if ((rc = new_blockset(B, H, nB, block, LBSA_SCOPE_ROUTED, p, s, &bs)) != LBSA_OK) return rc;
+  DeviceState* ds = nullptr;
+  Scratch ws;
+  if ((rc = device_state(&ds)) != LBSA_OK ||
+      (rc = scratch_alloc(ds, lbsa::select_routed_workspace_bytes(B, H, nB), s, &ws)) != LBSA_OK) {
+    lbsa_free(bs);
+    return rc;
+  }
+  cudaError_t e = lbsa::launch_select_routed(scores, B, H, nB, p, entropy_threshold, group, head_entropy, head_domain,
+                                             bs, ws.ptr, s);
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_select_routed launch");
   }
   *out = bs;
   return LBSA_OK;

@@ -53,13 +53,16 @@ __device__ __forceinline__ uint64_t threshold_T(uint64_t W, uint32_t Pfix) {
 
 // ---------------------------------------------------------------- row scope
 // One warp per row of nB scores; lane l holds elements l, l+32, ...
+// skip_head (NULL for plain row scope): rows of heads with skip_head[h] >= 0
+// (pooled heads of the routed scope) are left to the domain kernel.
 template <int EPL>
 __global__ void select_row_kernel(const float* __restrict__ scores, int R, int nB, uint32_t Pfix, int keep_all,
                                   int32_t* __restrict__ counts, int32_t* __restrict__ cols,
-                                  int32_t* __restrict__ status) {
+                                  int32_t* __restrict__ status, const int32_t* __restrict__ skip_head) {
   const int lane = threadIdx.x & 31;
   const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (row >= R) return;
+  if (skip_head && skip_head[row / nB] >= 0) return;      // warp-uniform
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
   int32_t* out = cols + row * nB;
   uint32_t bits[EPL];
@@ -660,9 +663,279 @@ __global__ void __launch_bounds__(256) head_floor_kernel(const int32_t* __restri
   }
 }
 
+// ---------------------------------------------------------------- routed scope
+// EG-Sparse abstract (readsearch.ai page of arXiv 2610.14672, "Competition
+// Domains Matter"): heads whose scores have low entropy compete in a pool
+// shared by a group of heads, the others keep per-row selection.
+//   head entropy  mean over the head's rows of the entropy of the row's
+//                 normalised scores, divided by ln(nB); a head is routed when
+//                 it is below the threshold; routed heads form consecutive
+//                 groups of `group` in head order
+//   domain        a pool's members' row i (flat index m*nB + j, m the member's
+//                 rank), or one high-entropy head's row i; each domain takes
+//                 the fixed-point threshold rule above.
+// High-entropy heads go through the row kernel (a one-head domain is a row);
+// the pools go through domain_select_kernel.  Pool table of batch element b
+// (int32, 2H + 2 entries): [0] = pool count np, [1 .. np + 1] = member
+// offsets, [H + 2 ..] = member heads.
+
+// Row entropy ln S - (sum_j x_j ln x_j) / S, S = sum_j x_j, in fp64 from fp32
+// logarithms (0 ln 0 = 0; a zero row gives 0; invalid scores give NaN or a
+// value the domain kernel rejects).  One warp per row, 8 rows per CTA; the CTA
+// writes the sum of its rows' entropies (fixed reduction order throughout, so
+// the result does not vary from run to run).  grid (ceil(nQ / 8), B*H).
+constexpr int kEntRowsPerCta = 8;
+__global__ void __launch_bounds__(256) row_entropy_kernel(const float* __restrict__ scores, int nQ, int nB,
+                                                          double* __restrict__ part) {
+  __shared__ double wsum[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.y, i = blockIdx.x * kEntRowsPerCta + warp;
+  double h = 0.0;
+  if (i < nQ) {                               // warp-uniform
+    const float* x = scores + (static_cast<long long>(g) * nQ + i) * nB;
+    double S = 0.0, L = 0.0;
+    for (int j = lane; j < nB; j += 32) {
+      const float v = __ldg(x + j);
+      if (v != 0.0f) {
+        S += v;
+        L += static_cast<double>(v) * static_cast<double>(logf(v));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      L += __shfl_xor_sync(0xffffffffu, L, o);
+    }
+    h = (S == 0.0) ? 0.0 : log(S) - L / S;   // lane 0's value is the one used
+  }
+  if (lane == 0) wsum[warp] = h;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s += wsum[u];
+    part[static_cast<long long>(g) * gridDim.x + blockIdx.x] = s;
+  }
+}
+
+// One CTA (256 threads) per batch element: head entropies (warp per head,
+// fixed order over the row-entropy partials), then the domain table; optional
+// caller copies of both.
+__global__ void __launch_bounds__(256) route_kernel(const double* __restrict__ part, int n_part, int H, int nQ, int nB,
+                                                    double threshold, int group, int32_t* __restrict__ dom,
+                                                    int32_t* __restrict__ head_dom, double* __restrict__ ent_out,
+                                                    int32_t* __restrict__ dom_out) {
+  extern __shared__ double sh_ent[];          // [H]
+  const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const double inv = (nB > 1) ? 1.0 / (static_cast<double>(nQ) * log(static_cast<double>(nB))) : 0.0;
+  for (int h = warp; h < H; h += 8) {
+    const double* r = part + (static_cast<long long>(b) * H + h) * n_part;
+    double s = 0.0;
+    for (int c = lane; c < n_part; c += 32) s += r[c];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) {
+      const double e = s * inv;
+      sh_ent[h] = e;
+      if (ent_out) ent_out[static_cast<long long>(b) * H + h] = e;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  int32_t* D = dom + static_cast<long long>(b) * (2 * H + 2);
+  int32_t* off = D + 1;
+  int32_t* mem = D + H + 2;
+  int nd = 0, nm = 0, rank = 0;
+  for (int h = 0; h < H; ++h) {               // routed heads, `group` to a pool, in head order (NaN is not below)
+    const bool routed = sh_ent[h] < threshold;
+    const int32_t id = routed ? rank / group : -1;
+    if (routed) {
+      if (rank % group == 0) off[nd++] = nm;
+      mem[nm++] = h;
+      ++rank;
+    }
+    head_dom[static_cast<long long>(b) * H + h] = id;
+    if (dom_out) dom_out[static_cast<long long>(b) * H + h] = id;
+  }
+  off[nd] = nm;
+  D[0] = nd;
+}
+
+// Sum over the CTA's 8 warps of a per-thread value below 2^54; uniform result.
+__device__ __forceinline__ unsigned long long cta_sum_u64(unsigned long long v, unsigned long long (*red)[8],
+                                                          int& parity) {
+  const unsigned long long ws = warp_sum_u64(v);
+  if ((threadIdx.x & 31) == 0) red[parity][threadIdx.x >> 5] = ws;
+  __syncthreads();
+  unsigned long long s = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) s += red[parity][u];
+  parity ^= 1;                                // the next sum writes the other buffer
+  return s;
+}
+
+// One CTA (256 threads) per (query block i, pool d, batch element b): the
+// pool's M*nB scores are staged in shared memory, the threshold bits tb are
+// found by a weighted radix select over the 30 significant bits in three
+// 10-bit digits (exact 64-bit bin sums in shared memory), then every member
+// row is emitted with the ties at tb ranked across the domain in flat order.
+__global__ void __launch_bounds__(256) domain_select_kernel(const float* __restrict__ scores, int H, int nQ, int nB,
+                                                            const int32_t* __restrict__ dom, uint32_t Pfix,
+                                                            int keep_all, int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ cols, int32_t* __restrict__ status) {
+  extern __shared__ uint32_t sbits[];         // [M * nB], then M + 1 tie offsets
+  __shared__ unsigned long long hist[kBins];
+  __shared__ unsigned long long red[2][8];
+  __shared__ uint32_t red_max[8];
+  __shared__ unsigned long long s_above;
+  __shared__ uint32_t s_prefix;
+  const int i = blockIdx.x, d = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* D = dom + static_cast<long long>(b) * (2 * H + 2);
+  if (d >= D[0]) return;                      // CTA-uniform
+  const int m0 = D[1 + d], M = D[2 + d] - m0;
+  const int32_t* mem = D + H + 2 + m0;
+  const int n = M * nB;
+  int32_t* tie_off = reinterpret_cast<int32_t*>(sbits + n);
+  unsigned long long wsum = 0;
+  uint32_t mx = 0;
+  int bad = 0;
+  for (int m = 0; m < M; ++m) {
+    const uint32_t* x =
+        reinterpret_cast<const uint32_t*>(scores) + ((static_cast<long long>(b) * H + mem[m]) * nQ + i) * nB;
+    for (int j = threadIdx.x; j < nB; j += blockDim.x) {
+      const uint32_t v = __ldg(x + j);
+      sbits[m * nB + j] = v;
+      if (v >= kInvalidBits) {
+        bad = 1;
+      } else {
+        wsum += fixed_weight(v);
+        mx = max(mx, v);
+      }
+    }
+  }
+  int parity = 0;
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) red_max[warp] = mx;
+  const int any_bad = __syncthreads_or(bad);
+  const unsigned long long W = cta_sum_u64(wsum, red, parity);
+  mx = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mx = max(mx, red_max[u]);
+  if (any_bad || keep_all) {
+    if (any_bad && threadIdx.x == 0) raise_status(status, LBSA_ERR_INVALID_SCORES);
+    for (int m = warp; m < M; m += 8) {
+      const long long r = (static_cast<long long>(b) * H + mem[m]) * nQ + i;
+      for (int j = lane; j < nB; j += 32) cols[r * nB + j] = j;
+      if (lane == 0) counts[r] = nB;
+    }
+    return;
+  }
+  const unsigned long long T = threshold_T(W, Pfix);
+  uint32_t tb, need;
+  if (T == 0) {
+    tb = mx;                                  // keep one pair: the highest score, lowest flat index
+    need = 1;
+  } else {
+    if (threadIdx.x == 0) {
+      s_above = 0;
+      s_prefix = 0;
+    }
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = 20 - kDigitBits * pass;
+#pragma unroll
+      for (int u = 0; u < kBins / 256; ++u) hist[threadIdx.x + 256 * u] = 0ull;
+      __syncthreads();                        // bins cleared; s_prefix / s_above of the last pass visible
+      const uint32_t prefix = s_prefix;
+      const unsigned long long above = s_above;
+      // the scores of one row mostly share their high digits: the lanes of a
+      // warp that hit the same bin first add their weights exactly (27 low
+      // bits and the rest, each total < 2^32) and one of them does the atomic
+      for (int e0 = threadIdx.x - lane; e0 < n; e0 += blockDim.x) {   // warp-uniform trip count
+        const int e = e0 + lane;
+        const uint32_t v = (e < n) ? sbits[e] : 0u;
+        const unsigned long long w = (e < n) ? fixed_weight(v) : 0ull;
+        const bool in = w != 0ull && (pass == 0 || (v >> (shift + kDigitBits)) == prefix);
+        const uint32_t bin = in ? ((v >> shift) & (kBins - 1)) : static_cast<uint32_t>(kBins);
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        const uint32_t lo = __reduce_add_sync(peers, static_cast<uint32_t>(w) & ((1u << 27) - 1u));
+        const uint32_t hi = __reduce_add_sync(peers, static_cast<uint32_t>(w >> 27));
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (static_cast<unsigned long long>(hi) << 27) + lo);
+      }
+      __syncthreads();
+      // thread t owns bins 4t .. 4t+3: suffix sums S[k] = weight of bins >= 4t + k
+      unsigned long long hv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) hv[k] = hist[4 * threadIdx.x + k];
+      unsigned long long x = (hv[0] + hv[1]) + (hv[2] + hv[3]);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+      }
+      if (lane == 0) red[parity][warp] = x;
+      __syncthreads();
+      unsigned long long later = 0;
+      for (int u = warp + 1; u < 8; ++u) later += red[parity][u];
+      parity ^= 1;
+      unsigned long long S[5];
+      S[0] = x + later;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) S[k + 1] = S[k] - hv[k];
+      // the largest bin with above + S(bin) >= T (it exists: the prefix's elements reach T - above);
+      // every thread read prefix / above before the binning barrier, so they may change now
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (above + S[k] >= T && above + S[k + 1] < T) {
+          s_prefix = (prefix << kDigitBits) | static_cast<uint32_t>(4 * threadIdx.x + k);
+          s_above = above + S[k + 1];
+        }
+      }
+    }
+    __syncthreads();
+    tb = s_prefix;
+    const unsigned long long ww = fixed_weight(tb);   // > 0: the chosen bin holds weight
+    need = static_cast<uint32_t>((T - s_above + ww - 1) / ww);
+  }
+  // ties at tb per member, then their exclusive offsets in flat order
+  for (int m = warp; m < M; m += 8) {
+    int c = 0;
+    for (int j = lane; j < nB; j += 32) c += (sbits[m * nB + j] == tb);
+    c = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+    if (lane == 0) tie_off[m + 1] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tie_off[0] = 0;
+    for (int m = 0; m < M; ++m) tie_off[m + 1] += tie_off[m];
+  }
+  __syncthreads();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int m = warp; m < M; m += 8) {
+    const long long r = (static_cast<long long>(b) * H + mem[m]) * nQ + i;
+    int32_t* out = cols + r * nB;
+    uint32_t ties_before = static_cast<uint32_t>(tie_off[m]);
+    int base = 0;
+    for (int j0 = 0; j0 < nB; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t v = (j < nB) ? sbits[m * nB + j] : 0u;
+      const bool tie = (j < nB) && v == tb;
+      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+      const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+      const bool keep = (j < nB) && (v > tb || (tie && rank < need));
+      const uint32_t kmask = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[base + __popc(kmask & lt_mask)] = j;
+      base += __popc(kmask);
+      ties_before += __popc(tmask);
+    }
+    if (lane == 0) counts[r] = base;
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s) {
+cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s,
+                              const int32_t* skip_head) {
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
   // two warps (rows) per block: residency is then bounded by registers, not by
@@ -671,7 +944,8 @@ cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa
   const long long blocks = (static_cast<long long>(R) * 32 + threads - 1) / threads;
   dim3 grid(static_cast<unsigned>(blocks));
 #define LBSA_SEL(EPL)                                                                                       \
-  select_row_kernel<EPL><<<grid, threads, 0, s>>>(scores, R, nB, P, keep_all, bs->counts, bs->cols, bs->status)
+  select_row_kernel<EPL><<<grid, threads, 0, s>>>(scores, R, nB, P, keep_all, bs->counts, bs->cols, bs->status, \
+                                                  skip_head)
   if (nB <= 32) LBSA_SEL(1);
   else if (nB <= 64) LBSA_SEL(2);
   else if (nB <= 128) LBSA_SEL(4);
@@ -764,6 +1038,38 @@ cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int 
   const int nQB = (nQ + 63) / 64;
   token_emit_kernel<<<static_cast<unsigned>(G) * nQB, 256, 0, s>>>(scores, G, nQ, nB, st, tie, bs->counts, bs->cols,
                                                                   bs->masks);
+  return cudaGetLastError();
+}
+
+size_t select_routed_workspace_bytes(int B, int H, int nB) {
+  const size_t parts = static_cast<size_t>(B) * H * ((nB + kEntRowsPerCta - 1) / kEntRowsPerCta);
+  return parts * sizeof(double) + static_cast<size_t>(B) * (3 * H + 2) * sizeof(int32_t) + 256;
+}
+
+size_t select_routed_smem_bytes(int H, int nB, int group) {
+  const int M = group < H ? group : H;
+  return static_cast<size_t>(M) * nB * sizeof(uint32_t) + static_cast<size_t>(M + 1) * sizeof(int32_t);
+}
+
+cudaError_t launch_select_routed(const float* scores, int B, int H, int nB, double p, double threshold, int group,
+                                 double* ent_out, int32_t* dom_out, lbsa_blockset* bs, void* ws, cudaStream_t s) {
+  const int n_part = (nB + kEntRowsPerCta - 1) / kEntRowsPerCta;
+  double* part = reinterpret_cast<double*>(ws);
+  int32_t* head_dom = reinterpret_cast<int32_t*>(part + static_cast<size_t>(B) * H * n_part);
+  int32_t* dom = head_dom + static_cast<size_t>(B) * H;
+  row_entropy_kernel<<<dim3(n_part, B * H), 256, 0, s>>>(scores, nB, nB, part);
+  route_kernel<<<B, 256, static_cast<size_t>(H) * sizeof(double), s>>>(part, n_part, H, nB, nB, threshold, group, dom,
+                                                                      head_dom, ent_out, dom_out);
+  cudaError_t e = launch_select_row(scores, B * H * nB, nB, p, bs, s, head_dom);
+  if (e != cudaSuccess) return e;
+  const size_t smem = select_routed_smem_bytes(H, nB, group);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(domain_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int max_pools = (H + group - 1) / group;
+  domain_select_kernel<<<dim3(nB, max_pools, B), 256, smem, s>>>(scores, H, nB, nB, dom, fixed_p(p),
+                                                                 p >= 1.0 ? 1 : 0, bs->counts, bs->cols, bs->status);
   return cudaGetLastError();
 }
 

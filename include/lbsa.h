@@ -63,7 +63,7 @@ typedef enum {
 
 typedef enum { LBSA_BF16 = 0, LBSA_F32 = 1 } lbsa_dtype;
 typedef enum { LBSA_SCORE_EXACT_MASS = 0, LBSA_SCORE_MEANPOOL = 1, LBSA_SCORE_MEANPOOL_TOKEN = 2 } lbsa_score_mode;
-typedef enum { LBSA_SCOPE_ROW = 0, LBSA_SCOPE_HEAD = 1, LBSA_SCOPE_TOKEN = 2 } lbsa_scope;
+typedef enum { LBSA_SCOPE_ROW = 0, LBSA_SCOPE_HEAD = 1, LBSA_SCOPE_TOKEN = 2, LBSA_SCOPE_ROUTED = 3 } lbsa_scope;
 typedef enum {
   LBSA_PART_RASTER = 0,         /* identity                                        */
   LBSA_PART_1D = 1,             /* temporal rows: t fastest                        */
@@ -189,6 +189,45 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
  * pair of the head and set LBSA_ERR_INVALID_SCORES.  Scratch: the radix
  * histograms and per-token tie counts of B*H heads, from the library pool. */
 int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_valid, int32_t block, double p,
+                       lbsa_blockset** out, void* stream);
+
+/* Stage 2 with entropy-routed competition domains (EG-Sparse abstract,
+ * readsearch.ai page of arXiv 2610.14672, "Competition Domains Matter:
+ * Selective Head Globalization for Training-Free Sparse Attention in Video
+ * Diffusion Transformers": low-entropy heads compete in a grouped cross-head
+ * pool, high-entropy heads keep per-row selection, from the scores already
+ * materialised).  Into a new blockset (scope LBSA_SCOPE_ROUTED, row lists as
+ * LBSA_SCOPE_ROW).
+ *   scores   fp32 [B, H, nB, nB] contiguous device array, 0 <= x < 2
+ *   block    tokens per block the scores were computed with (64 or 128)
+ *   p        threshold in (0, 1]; p = 1 keeps every block
+ *   entropy_threshold  head (b, h) is routed when its entropy E < this value
+ *            (any non-NaN value; <= 0 routes none, > 1 routes all)
+ *   group    >= 1: routed heads of one batch element, in ascending head
+ *            order, form consecutive pools of `group` heads (the last may be
+ *            smaller); group >= H makes one pool of all routed heads
+ *   head_entropy  optional out (NULL to skip): device fp64 [B, H], E of
+ *            every head
+ *   head_domain   optional out (NULL to skip): device int32 [B, H], -1 for a
+ *            head selected per row, else its pool's index within b
+ *   out      receives a new blockset (free with lbsa_free).
+ * E = (1 / (nB ln nB)) sum_i H_i with H_i = ln S_i - (sum_j x_ij ln x_ij) / S_i,
+ * S_i = sum_j x_ij, the entropy of row i's normalised scores (0 ln 0 = 0; a
+ * zero row gives 0; nB = 1 gives E = 0), computed from fp32 logarithms in fp64
+ * (absolute error a few 1e-7).  Domains: a high-entropy head's row i, or a
+ * pool's member rows i, flat index m*nB + j with m the member's rank in the
+ * pool.  Every domain takes the lbsa_select rule (exact fixed-point sums,
+ * score descending then flat index ascending, at least one pair); a member's
+ * row keeps the pairs of the prefix that are its own and may be empty (its
+ * attention output is then 0).  A domain holding a NaN, negative or >= 2
+ * score keeps every block of its rows and sets LBSA_ERR_INVALID_SCORES (a
+ * head with a NaN or negative score has a NaN entropy and is never routed).
+ * Scratch: B*H*ceil(nB/8) fp64 partial entropy sums and the domain tables,
+ * from the library pool; nB <= 1024, H <= 4096 and B*H <= 65535; a pool's
+ * min(group, H) * nB scores must fit 200 KiB of shared memory, else
+ * LBSA_ERR_UNSUPPORTED. */
+int lbsa_select_routed(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,
+                       double entropy_threshold, int32_t group, double* head_entropy, int32_t* head_domain,
                        lbsa_blockset** out, void* stream);
 
 /* Stage 3: block-sparse attention over a (frozen) blockset.

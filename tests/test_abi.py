@@ -27,7 +27,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 15
     for n in names:
         assert hasattr(lib, n), n
-    assert lbsa.lbsa_version() == 100
+    assert lbsa.lbsa_version() == 101
 
 
 def _desc(**kw):
@@ -132,6 +132,34 @@ def test_select_tokens_rejects_bad_block_p_and_size():
     assert lib.lbsa_select_tokens(p, 0, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.25, None, None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(None, 1, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+def test_select_routed_rejects_bad_args():
+    lib = lbsa.load_library()
+    buf = np.zeros(4096, dtype=np.float32)                  # host memory: rejected before any launch
+    h = ctypes.c_void_p()
+    p = ctypes.c_void_p(buf.ctypes.data)
+    ok = dict(B=1, H=4, nB=8, block=64, p=0.9, thr=0.5, group=2)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return lib.lbsa_select_routed(a.get("ptr", p), a["B"], a["H"], a["nB"], a["block"], a["p"], a["thr"],
+                                      a["group"], None, None, a.get("out", ctypes.byref(h)), None)
+
+    assert call(block=32) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert call(p=0.0) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(p=1.5) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(p=float("nan")) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(thr=float("nan")) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(group=0) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(B=0) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(B=20, H=4000) == lbsa.LBSA_ERR_UNSUPPORTED                # B*H > 65535
+    assert call(nB=1025, group=1) == lbsa.LBSA_ERR_UNSUPPORTED             # past the row kernel's width
+    assert call(H=4097) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert call(H=64, nB=1024, group=64) == lbsa.LBSA_ERR_UNSUPPORTED   # a 64-head pool of 1024 blocks: 256 KiB
+    assert call(out=None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert call(ptr=None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert "200 KiB" in (call(H=64, nB=1024, group=64) and lbsa.lbsa_last_error())
 
 
 def test_call_log_reports_calls_and_errors():
