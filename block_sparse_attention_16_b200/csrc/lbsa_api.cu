@@ -11,6 +11,7 @@
 #include <cudaTypedefs.h>
 
 #include "lbsa_device.cuh"
+#include "lbsa_routed.h"
 
 namespace {
 

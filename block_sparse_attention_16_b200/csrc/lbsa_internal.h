@@ -80,7 +80,7 @@ cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d
 
 // selection (select.cu)
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,
-                              cudaStream_t s, const int32_t* skip_head = nullptr);
+                              cudaStream_t s);
 cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int k, const int32_t* head_floor,
                                lbsa_blockset* bs, cudaStream_t s);
 cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, int n_valid, int32_t* head_floor,
@@ -93,14 +93,6 @@ cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double
 // bs->counts / cols / masks per query block
 cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int nB, double p, lbsa_blockset* bs,
                                  void* workspace, cudaStream_t s);
-// routed scope (entropy-routed competition domains): scratch = fp64 partial
-// sums of the row entropies ([B*H*ceil(nB/8)]) + per-head pool ids + pool
-// tables; dynamic shared memory of the pool kernel
-size_t select_routed_workspace_bytes(int B, int H, int nB);
-size_t select_routed_smem_bytes(int H, int nB, int group);
-cudaError_t launch_select_routed(const float* scores, int B, int H, int nB, double p, double threshold, int group,
-                                 double* ent_out, int32_t* dom_out, lbsa_blockset* bs, void* workspace,
-                                 cudaStream_t s);
 cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col,
                               int32_t* nnz_dev, cudaStream_t s);
 cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blockset* bs,

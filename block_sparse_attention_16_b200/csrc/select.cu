@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "lbsa_device.cuh"
+#include "lbsa_routed.h"
 
 namespace lbsa {
 namespace {
@@ -934,8 +935,9 @@ __global__ void __launch_bounds__(256) domain_select_kernel(const float* __restr
 
 }  // namespace
 
-cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s,
-                              const int32_t* skip_head) {
+// skip_head: see select_row_kernel (NULL for plain row scope)
+static cudaError_t launch_select_row_skip(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s,
+                                   const int32_t* skip_head) {
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
   // two warps (rows) per block: residency is then bounded by registers, not by
@@ -955,6 +957,10 @@ cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa
   else return cudaErrorInvalidValue;
 #undef LBSA_SEL
   return cudaGetLastError();
+}
+
+cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s) {
+  return launch_select_row_skip(scores, R, nB, p, bs, s, nullptr);
 }
 
 cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int k, const int32_t* head_floor,
@@ -1060,7 +1066,7 @@ cudaError_t launch_select_routed(const float* scores, int B, int H, int nB, doub
   row_entropy_kernel<<<dim3(n_part, B * H), 256, 0, s>>>(scores, nB, nB, part);
   route_kernel<<<B, 256, static_cast<size_t>(H) * sizeof(double), s>>>(part, n_part, H, nB, nB, threshold, group, dom,
                                                                       head_dom, ent_out, dom_out);
-  cudaError_t e = launch_select_row(scores, B * H * nB, nB, p, bs, s, head_dom);
+  cudaError_t e = launch_select_row_skip(scores, B * H * nB, nB, p, bs, s, head_dom);
   if (e != cudaSuccess) return e;
   const size_t smem = select_routed_smem_bytes(H, nB, group);
   if (smem > 48 * 1024) {
