@@ -14,6 +14,9 @@
  *      all block pairs of a head (VMoBA global selection).  The result is a
  *      blockset that can be frozen and reused by later calls (LoSA abstract:
  *      the frozen block indices are reused for all remaining steps).
+ *      Further rules: lbsa_select_rule (Local + TopK; top-p with a per-head
+ *      floor), lbsa_select_tokens (per-token pairs), lbsa_select_routed
+ *      (entropy-routed cross-head pools).
  *   3. lbsa_attend -- block-sparse flash attention that visits only the kept
  *      key blocks (VMoBA review: only the selected blocks contribute their
  *      actual key-value pairs).
