@@ -55,17 +55,26 @@ def attention_flops(counts, nB, block, n_valid, d):
     """4*d*sum over kept (query block, key block) of valid_q * valid_k."""
     valid = np.full(nB, block, dtype=np.float64)
     valid[-1] = n_valid - (nB - 1) * block
-    c = counts.reshape(-1, nB, nB) if counts.ndim == 3 else counts
+    c = np.asarray(counts).reshape(-1, nB, nB)          # [G, nB, nB] or flat [G*nB, nB]
     return 4.0 * d * float(np.einsum("gij,i,j->", c, valid, valid))
 
 
 def token_flops(lbsa, bs, wl):
-    """Attention FLOPs on the kept (token, key block) pairs of a per-token blockset,
-    4*d*sum over tokens of their kept blocks' valid keys; also the kept-pair
-    density and the fraction of tokens that keep nothing."""
+    """token_flops_of on a per-token blockset's device arrays."""
     counts, cols = (x.cpu().numpy() for x in lbsa.lbsa_blockset_views(bs))
     masks = lbsa.lbsa_blockset_masks(bs).cpu().numpy().view(np.uint64)
+    return token_flops_of(counts, cols, masks, wl)
+
+
+def token_flops_of(counts, cols, masks, wl):
+    """Attention FLOPs on the kept (token, key block) pairs of a per-token blockset
+    (counts [R], cols and masks [R, nB] as the library lays them out), 4*d*sum
+    over tokens of their kept blocks' valid keys; also the kept-pair density and
+    the fraction of tokens that keep nothing."""
     nB, blk = wl.n_blocks, wl.block
+    counts = np.asarray(counts).reshape(-1)
+    cols = np.asarray(cols).reshape(-1, nB)
+    masks = np.asarray(masks, dtype=np.uint64).reshape(-1, nB)
     valid = np.full(nB, blk, dtype=np.float64)
     valid[-1] = wl.n_valid - (nB - 1) * blk
     slot = np.arange(nB)[None, :] < counts[:, None]
