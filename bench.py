@@ -91,6 +91,16 @@ def token_flops_of(counts, cols, masks, wl):
     return fl, kept / (n_tok * nB), 1.0 - float(has) / n_tok
 
 
+def median_entropy(ent):
+    """Routing threshold of the entropy-routed sweep lines: the median of one batch
+    element's head entropies (mean of the two middle values for an even count), so
+    that the heads strictly below it (half of them when the values are distinct) are
+    pooled."""
+    e = np.sort(np.asarray(ent.cpu() if hasattr(ent, "cpu") else ent, dtype=np.float64).reshape(-1))
+    n = e.shape[0]
+    return float(e[n // 2]) if n % 2 else float((e[n // 2 - 1] + e[n // 2]) / 2)
+
+
 def kept_mask(row_ptr, col, rows, nB):
     m = np.zeros((rows, nB), dtype=np.float64)
     r = np.repeat(np.arange(rows), np.diff(row_ptr))
@@ -468,8 +478,7 @@ def run_profile(kernel):
         qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
         sc = lbsa.lbsa_score(qp, kp, wl.block)
         _, ent, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, -1.0, 1)
-        e_sorted = ent[0].sort().values
-        thr = float((e_sorted[wl.H // 2 - 1] + e_sorted[wl.H // 2]) / 2)
+        thr = median_entropy(ent[0])
         for _ in range(2):
             bs, _, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, thr, 3)
         lbsa.lbsa_attend(qp, kp, vp, bs)
@@ -630,8 +639,7 @@ def run_sweep(args):
     # entropy pooled `group` at a time, the rest per row, p = 0.99; and the
     # all-head pool of the abstract's diagnostic (every head routed, one pool)
     _, ent, _ = lbsa.lbsa_select_routed(sc, wl.block, 0.99, -1.0, 1)
-    e_sorted = ent[0].sort().values
-    thr = float((e_sorted[wl.H // 2 - 1] + e_sorted[wl.H // 2]) / 2)
+    thr = median_entropy(ent[0])
     for thr_, group in ((thr, 3), (thr, 6), (thr, wl.H), (2.0, wl.H)):
         bs, _, dom = lbsa.lbsa_select_routed(sc, wl.block, 0.99, thr_, group)
         fl, m = flops_of(bs, wl)

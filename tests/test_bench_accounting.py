@@ -100,3 +100,11 @@ def test_token_flops_closed_forms():
     assert fl == 4.0 * wl.d * wl.n_valid ** 2 and dens == 1.0 and empty == 0.0
     nothing = np.zeros((1, wl.n_valid, nB), dtype=bool)
     assert bench.token_flops_of(*_token_layout(nothing, wl), wl) == (0.0, 0.0, 1.0)
+
+
+def test_median_entropy_threshold():
+    assert bench.median_entropy(np.array([0.9, 0.1, 0.5, 0.3])) == 0.4
+    assert bench.median_entropy(np.array([0.9, 0.1, 0.5])) == 0.5
+    e = np.array([0.39, 0.94, 0.52, 0.83, 0.70, 0.41, 0.9998, 0.9995, 0.9998, 0.9998, 0.9995, 0.9997])
+    thr = bench.median_entropy(e)
+    assert (e < thr).sum() == 6                           # half the heads pooled
