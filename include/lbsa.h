@@ -197,9 +197,9 @@ int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_vali
 /* Stage 2 with entropy-routed competition domains (EG-Sparse abstract,
  * readsearch.ai page of arXiv 2610.14672, "Competition Domains Matter:
  * Selective Head Globalization for Training-Free Sparse Attention in Video
- * Diffusion Transformers": low-entropy heads compete in a grouped cross-head
- * pool, high-entropy heads keep per-row selection, from the scores already
- * materialised).  Into a new blockset (scope LBSA_SCOPE_ROUTED, row lists as
+ * Diffusion Transformers": heads whose scores have low entropy select jointly
+ * with a group of other heads, the rest per row, from the block scores the
+ * path computes anyway).  Into a new blockset (scope LBSA_SCOPE_ROUTED, row lists as
  * LBSA_SCOPE_ROW).
  *   scores   fp32 [B, H, nB, nB] contiguous device array, 0 <= x < 2
  *   block    tokens per block the scores were computed with (64 or 128)

@@ -17,9 +17,9 @@ computes, written from the pages' prose:
     "Local + TopK" selection of the training-free experiments.
   * SCOPE (abstract, mlsift.com): hybrid Top-p with a head-specific Top-k
     floor from the size-weighted mean of the initially retained counts.
-  * EG-Sparse (abstract, readsearch.ai page of arXiv 2610.14672): low-entropy
-    heads routed to a grouped cross-head pool, per-row selection for the
-    high-entropy heads, from the scores already materialised.
+  * EG-Sparse (abstract, readsearch.ai page of arXiv 2610.14672): heads whose
+    scores have low entropy select jointly with a group of other heads, the
+    rest per row, using only the block scores computed anyway.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  It imports nothing from the CUDA library or its

@@ -4,9 +4,9 @@ EG-Sparse abstract (readsearch.ai page of arXiv 2610.14672, "Competition
 Domains Matter: Selective Head Globalization for Training-Free Sparse
 Attention in Video Diffusion Transformers"): the usual block selection lets
 the key blocks of one query row of one head compete; EG-Sparse routes the
-heads whose scores have low entropy to a cross-head pool shared by a group of
-heads, keeps per-row selection for the high-entropy heads, and uses only the
-scores the sparse pipeline has already materialised.
+heads whose scores have low entropy to a pool shared by a group of heads,
+keeps per-row selection for the other heads, and needs nothing beyond the block
+scores the sparse path computes anyway.
 
 The abstract fixes neither the entropy, the routing rule, the grouping nor
 the rule inside a pool.  Readings taken here, each the plainest one the rest
