@@ -1,8 +1,8 @@
 // Block-sparse flash attention on sm_100a tensor cores (bf16 in, fp32 accumulate).
 //
 // What it computes (VMoBA review on pith.science, "What carries the argument":
-// only the selected key blocks contribute their actual key-value pairs; LoSA
-// abstract: the frozen block indices are reused at every later step):
+// attention runs on the true keys and values of the kept blocks and on nothing
+// else; LoSA abstract: the frozen block indices are reused at every later step):
 //   out_r = sum_{c in K_i} softmax_{c in K_i}(q_r . k_c / sqrt(d)) v_c
 // where K_i is the set of valid keys of the blocks kept for query block i.
 // An empty list gives out_r = 0 and lse_r = -inf.

@@ -1,6 +1,6 @@
 // Block-mean proxy scores (VMoBA review on pith.science, arXiv 2506.23858,
-// "What carries the argument": every key block is represented by its mean key
-// and queries score these block means).  Block-granular reading: the query
+// "What carries the argument": each key block stands in as the mean of its
+// keys, and queries score those means).  Block-granular reading: the query
 // side is pooled the same way, and the similarities of one head are
 // normalised by a softmax over all of its query-block x key-block pairs:
 //   qbar_i = mean_{r in I_i} q_r,  kbar_j = mean_{c in J_j} k_c   (fp32)
@@ -9,9 +9,8 @@
 // Three kernels: block means (reads Q and K once, 16-byte loads), the 64x64
 // tiles of s with per-tile (max, sum of exp), and the normalisation.
 //
-// Per-token mode (the same review: every query token scores the key-block
-// means, "full query-by-block similarity matrix", referee report major
-// comment 1):
+// Per-token mode (the same review, referee report major comment 1: every
+// query token against every key-block mean):
 //   s_rj = q_r . kbar_j / sqrt(d),   score[b,h,r,j] = exp(s_rj - M) / Z
 // over the head's n_valid x nB (token, key block) pairs; the logits kernel
 // then reads its rows straight from Q instead of from the query-block means.

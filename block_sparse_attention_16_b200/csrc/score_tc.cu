@@ -1,7 +1,7 @@
 // Exact block attention mass on sm_100a tensor cores (bf16 in, fp32 out).
 //
-// LoSA (abstract, scholarbro.com author page of C. Sun) measures the exact
-// block attention masses at one dense step.  Reading used for how the rows of a
+// LoSA (abstract, scholarbro.com author page of C. Sun) takes the block masses
+// exactly, from a single dense step.  Reading used for how the rows of a
 // query block combine: the mean over the block's valid rows, so
 //   mass[b,h,i,j] = (1/|I_i|) sum_{r in I_i} sum_{c in J_j} softmax_c(q_r.k_c/sqrt(d)).
 //

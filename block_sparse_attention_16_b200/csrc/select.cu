@@ -1,8 +1,9 @@
-// Mass-threshold block selection (LoSA abstract: per head and query block, the
-// smallest key/value block set whose retained mass meets the threshold; VMoBA
-// review on pith.science, circularity check: the smallest k' whose cumulative
-// normalized similarity reaches tau, with VMoBA's global selection over all
-// block pairs of a head, where query rows may come out empty).
+// Mass-threshold block selection (LoSA abstract: per head and query block, as
+// few key/value blocks as retain the threshold share of the mass; VMoBA
+// review on pith.science, circularity check: the least count k' of pairs whose
+// running sum of normalised similarity gets to tau, with VMoBA's global
+// selection over all block pairs of a head, where query rows may come out
+// empty).
 //
 // The cumulative sum is exact so that the kept set does not depend on the
 // order of a parallel reduction:

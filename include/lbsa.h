@@ -9,8 +9,9 @@
  *      pith.science, arXiv 2506.23858, "What carries the argument").
  *   2. lbsa_select -- mass-threshold selection: sort the scores, accumulate,
  *      keep the smallest key-block set whose retained mass reaches p (LoSA
- *      abstract; VMoBA review, circularity check: smallest k' whose cumulative
- *      normalized similarity reaches tau), per query-block row (LoSA) or over
+ *      abstract; VMoBA review, circularity check: the least count k' of pairs
+ *      whose running sum of normalised similarity gets to tau), per
+ *      query-block row (LoSA) or over
  *      all block pairs of a head (VMoBA global selection).  The result is a
  *      blockset that can be frozen and reused by later calls (LoSA abstract:
  *      the frozen block indices are reused for all remaining steps).
@@ -18,8 +19,8 @@
  *      floor), lbsa_select_tokens (per-token pairs), lbsa_select_routed
  *      (entropy-routed cross-head pools).
  *   3. lbsa_attend -- block-sparse flash attention that visits only the kept
- *      key blocks (VMoBA review: only the selected blocks contribute their
- *      actual key-value pairs).
+ *      key blocks (VMoBA review: attention runs on the true keys and values of
+ *      the kept blocks and nothing else).
  * plus lbsa_permute / lbsa_partition_perm for the 1D / 2D / 3D block
  * partitions of the token grid (VMoBA review: layer-wise cyclic 1D-2D-3D
  * partition).
@@ -91,8 +92,8 @@ typedef struct lbsa_blockset lbsa_blockset;
 
 /* Stage 1: block scores.
  * LoSA abstract (exact mass) / VMoBA review "What carries the argument"
- * (block-mean proxy; per-token queries: referee report major comment 1, "full
- * query-by-block similarity matrix").
+ * (block-mean proxy; per-token queries: referee report major comment 1, every
+ * query token against every key-block mean).
  *   q, k    [B, H, N_valid, d] per desc (bf16 or fp32)
  *   block   tokens per block, 64 or 128 (same for queries and keys)
  *   mode    LBSA_SCORE_EXACT_MASS: scores[b,h,i,j] = mean over the valid
@@ -157,9 +158,9 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
  *       training-free experiments select blocks by "Local + TopK", with
  *       k = 2, 6 or 18).  Row (b, h, i) keeps its own key block i plus the k
  *       top-ranked other key blocks: min(k + 1, nB) blocks.  p, n_valid unused.
- *   LBSA_RULE_TOPP_FLOOR  SCOPE abstract (a head-specific Top-k from the
- *       query-size-weighted mean of the initially retained key counts; extra
- *       keys only where the initial count falls below it).  The
+ *   LBSA_RULE_TOPP_FLOOR  SCOPE abstract (a per-head Top-k set to the mean
+ *       of the key counts the first pass kept, weighted by query-cluster size;
+ *       more keys only where a count is below it).  The
  *       LBSA_SCOPE_ROW threshold rule with p gives counts c_i; the head's
  *       floor is K = ceil(sum_i v_i c_i / sum_i v_i) with v_i the valid tokens
  *       of query block i, min(block, n_valid - i * block); row i keeps the

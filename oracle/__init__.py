@@ -3,20 +3,20 @@
 Plain, slow, fp64 NumPy restatement of what the block-sparse attention path
 computes, written from the pages' prose:
 
-  * LoSA (abstract, scholarbro.com author page of C. Sun): exact block
-    attention mass measured at one dense step; per head and query block the
-    smallest key/value block set whose retained mass meets a 99% threshold;
-    the frozen block indices reused at later steps.
+  * LoSA (abstract, scholarbro.com author page of C. Sun): block masses
+    measured exactly during one dense step; per head and query block as few
+    key/value blocks as keep 99% of the mass; the same block indices
+    reused, frozen, at later steps.
   * VMoBA (pith.science review of arXiv 2506.23858, "What carries the
     argument", referee report major comments 1-2, circularity check, free
-    parameters): key blocks represented by their mean, scored by query-block
-    means or by every query token; global selection over all query-key block
-    (or query-token, key-block) pairs of a head; threshold selection keeping the
-    smallest number of pairs whose cumulative normalized similarity reaches
-    tau; the layer-wise 1D-2D-3D block partition; empty query rows; the
-    "Local + TopK" selection of the training-free experiments.
-  * SCOPE (abstract, mlsift.com): hybrid Top-p with a head-specific Top-k
-    floor from the size-weighted mean of the initially retained counts.
+    parameters): each key block stands in as its mean key, scored by
+    query-block means or by every query token; one selection over all
+    query-key block (or query-token, key-block) pairs of a head; the least
+    count of pairs whose running sum of normalised similarity gets to tau; a
+    1D / 2D / 3D block partition that changes from layer to layer; empty query
+    rows; the "Local + TopK" selection of the training-free experiments.
+  * SCOPE (abstract, mlsift.com): hybrid Top-p with a per-head Top-k floor,
+    the size-weighted mean of the counts the first pass kept.
   * EG-Sparse (abstract, readsearch.ai page of arXiv 2610.14672): heads whose
     scores have low entropy select jointly with a group of other heads, the
     rest per row, using only the block scores computed anyway.

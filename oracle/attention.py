@@ -5,9 +5,9 @@ page): plain bidirectional softmax attention over the whole 3D token sequence,
 scale 1/sqrt(d) (the pages never state the scale; the mean-pooled proxy
 workload writes 1/sqrt(d), and it is the standard choice).
 
-Sparse attention follows the VMoBA review ("What carries the argument"): only
-the selected key blocks contribute their actual key-value pairs, and the
-softmax is renormalised over the union of their valid keys.  A query row whose
+Sparse attention follows the VMoBA review ("What carries the argument"):
+attention runs on the true keys and values of the kept blocks and nothing else,
+and the softmax is renormalised over the union of their valid keys.  A query row whose
 list is empty (possible under VMoBA's global selection, referee report major
 comment 1) attends to nothing: its output is 0 and its log-sum-exp is -inf.
 

@@ -12,8 +12,8 @@ row of the score matrix sums to 1:
 where I_i, J_j are the valid tokens (index < n_valid) of blocks i and j.
 
 meanpool_scores -- VMoBA's block-mean proxy (pith.science review of arXiv
-2506.23858, "What carries the argument"): each key block is represented by
-its mean key.  The pages score per-token queries against block means; the
+2506.23858, "What carries the argument"): each key block stands in as the
+mean of its keys.  The pages score per-token queries against block means; the
 block-granular reading used here scores the query-block mean instead:
 
     qbar_i = mean_{r in I_i} q_r,  kbar_j = mean_{c in J_j} k_c,
@@ -24,8 +24,8 @@ block-granular reading used here scores the query-block mean instead:
 over all query-block x key-block pairs of the head.
 
 token_meanpool_scores -- the same proxy in the pages' own granularity: every
-query token scores every key-block mean ("full query-by-block similarity
-matrix", referee report major comment 1), and the similarities of one head
+query token scores every key-block mean (the complete token-by-block score
+table of referee report major comment 1), and the similarities of one head
 are normalised by a softmax over all of its (query token, key block) pairs:
 
     s_rj = q_r . kbar_j / sqrt(d)      for valid tokens r < n_valid

@@ -1,8 +1,8 @@
 """Mass-threshold block selection (oracle; test infrastructure).
 
 Rule (LoSA abstract, scholarbro.com author page): per head and query block,
-keep the smallest key/value block set whose retained attention mass meets the
-threshold p (0.99 by default).  Rule (VMoBA review on pith.science,
+keep as few key/value blocks as retain at least the share p of the attention
+mass (0.99 by default).  Rule (VMoBA review on pith.science,
 circularity check and referee report): sort the normalized similarities of a
 head's query-key block pairs, keep the smallest count k' whose cumulative sum
 reaches tau (0.25), rows may end up empty.

@@ -9,11 +9,10 @@ key blocks of the row.  Ordering as in the threshold rule: fp32 score bits
 descending, then lower key-block index first.  Rows keep min(k + 1, nB)
 blocks.
 
-Top-p with a per-head floor (SCOPE abstract on mlsift.com: on top of hybrid
-Top-p / Top-k selection, a head-specific Top-k value is derived online by
-averaging the initially retained key counts within the head, weighted by
-query-cluster size, and extra keys are selected only for clusters whose
-initial count falls below it).  Block-level reading taken here:
+Top-p with a per-head floor (SCOPE abstract on mlsift.com: hybrid Top-p /
+Top-k selection whose Top-k is set per head while running, as the mean of the
+key counts the first pass kept in that head, each weighted by the size of its
+query cluster; only clusters that kept fewer than that receive more keys).  Block-level reading taken here:
   * initial counts c_i: the row-scope threshold rule of select.py (p);
   * weights: the valid tokens of query block i, v_i = min(block, n_valid - i*block);
   * floor K_h = ceil(sum_i v_i c_i / sum_i v_i), exact integer arithmetic;
