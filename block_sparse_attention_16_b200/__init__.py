@@ -134,6 +134,24 @@ def _desc(x: torch.Tensor, n_valid: int | None = None) -> _Desc:
     return _Desc(B, H, N if n_valid is None else n_valid, d, dt, 0, x.stride(0), x.stride(1), x.stride(2))
 
 
+def _on_device(x, name: str, dtype=None, min_numel: int = 0, contiguous: bool = True):
+    """The library reads and writes only device memory of the current CUDA
+    device: reject anything else before a pointer reaches it."""
+    if x is None:
+        return
+    if not isinstance(x, torch.Tensor) or not x.is_cuda:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if x.device.index != torch.cuda.current_device():
+        raise LbsaError(LBSA_ERR_INVALID_ARG,
+                        f"{name} lives on cuda:{x.device.index}, the current device is cuda:{torch.cuda.current_device()}")
+    if dtype is not None and x.dtype != dtype:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"{name} must be {dtype}, got {x.dtype}")
+    if contiguous and not x.is_contiguous():
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if x.numel() < min_numel:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"{name} holds {x.numel()} elements, {min_numel} needed")
+
+
 def _same_layout(a: torch.Tensor, b: torch.Tensor):
     if a.shape != b.shape or a.stride() != b.stride() or a.dtype != b.dtype or a.device != b.device:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "q, k, v (and out) must share shape, strides, dtype and device")
@@ -173,6 +191,8 @@ def lbsa_score(q, k, block: int, mode: str = "exact", scores=None, lse=None, wan
         scores = torch.empty(B, H, N if mode == "meanpool_token" else nB, nB, dtype=torch.float32, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
+    _on_device(scores, "scores", torch.float32)
+    _on_device(lse, "lse", torch.float32)
     _check(load_library().lbsa_score(_ptr(q), _ptr(k), ctypes.byref(desc), block, _MODES[mode],
                                      _ptr(scores), _ptr(lse), _stream(stream)))
     return (scores, lse) if (want_lse or lse is not None) else scores
@@ -180,6 +200,7 @@ def lbsa_score(q, k, block: int, mode: str = "exact", scores=None, lse=None, wan
 
 def lbsa_select(scores, block: int, p: float = 0.99, scope: str = "row", stream=None) -> Blockset:
     """Mass-threshold selection of fp32 scores [B, H, nB, nB] into a new blockset."""
+    _on_device(scores, "scores")
     if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, nB, nB] tensor")
     B, H, nB, nB2 = scores.shape
@@ -194,6 +215,7 @@ def lbsa_select(scores, block: int, p: float = 0.99, scope: str = "row", stream=
 def lbsa_select_tokens(scores, block: int = 64, p: float = 0.25, stream=None) -> Blockset:
     """Head-scope selection over the (query token, key block) pairs of fp32
     scores [B, H, N, nB] into a new per-token blockset (64-token blocks)."""
+    _on_device(scores, "scores")
     if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, N, nB] tensor")
     B, H, N, nB = scores.shape
@@ -252,6 +274,8 @@ def lbsa_score_attend(q, k, v, block: int, scores=None, out=None, lse=None, want
     if want_lse and lse is None:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
     desc = _desc(q)
+    _on_device(scores, "scores", torch.float32, B * H * nB * nB)
+    _on_device(lse, "lse", torch.float32, B * H * N)
     _check(load_library().lbsa_score_attend(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(desc), block, _ptr(scores),
                                             _ptr(out), _ptr(lse), _stream(stream)))
     return (scores, out, lse) if want_lse else (scores, out)
@@ -266,6 +290,7 @@ def lbsa_select_rule(scores, block: int, rule: str, n_valid: int, p: float = 0.9
     keeps each row's own key block plus the k top-ranked others; "topp_floor"
     applies the row threshold rule with p, then raises every row to its head's
     size-weighted mean count (rounded up)."""
+    _on_device(scores, "scores")
     if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, nB, nB] tensor")
     B, H, nB, nB2 = scores.shape
@@ -283,6 +308,7 @@ def lbsa_select_routed(scores, block: int, p: float, entropy_threshold: float, g
     in head order, and each pool's rows of one query block compete together;
     the other heads take the row rule.  Returns (blockset, head entropy fp64
     [B, H], head domain int32 [B, H]: -1 per row, else the pool index)."""
+    _on_device(scores, "scores")
     if scores.dtype != torch.float32 or not scores.is_contiguous() or scores.dim() != 4:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be a contiguous fp32 [B, H, nB, nB] tensor")
     B, H, nB, nB2 = scores.shape
@@ -307,6 +333,7 @@ def lbsa_attend(q, k, v, bs: Blockset, out=None, lse=None, want_lse=False, strea
     if want_lse and lse is None:
         lse = torch.empty(q.shape[0], q.shape[1], q.shape[2], dtype=torch.float32, device=q.device)
     desc = _desc(q)
+    _on_device(lse, "lse", torch.float32, q.shape[0] * q.shape[1] * q.shape[2])
     _check(load_library().lbsa_attend(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(desc), bs.handle,
                                       _ptr(out), _ptr(lse), _stream(stream)))
     return (out, lse) if (want_lse or lse is not None) else out
@@ -333,8 +360,20 @@ def lbsa_blockset_export(bs: Blockset, stream=None):
 
 
 def lbsa_blockset_from_csr(row_ptr, col, B: int, H: int, nB: int, block: int, stream=None) -> Blockset:
+    """Blockset from a CSR on the device (row_ptr [B*H*nB + 1], col [nnz]).  The
+    row pointers are checked here (start at 0, never decrease, end inside col),
+    since the library indexes col with them; column ids are checked on the
+    device (status word)."""
+    _on_device(row_ptr, "row_ptr", contiguous=False)
+    _on_device(col, "col", contiguous=False)
     row_ptr = row_ptr.to(torch.int32).contiguous()
     col = col.to(torch.int32).contiguous()
+    R = B * H * nB
+    if row_ptr.numel() != R + 1:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"row_ptr holds {row_ptr.numel()} entries, B*H*nB + 1 = {R + 1} needed")
+    rp = row_ptr.cpu()
+    if int(rp[0]) != 0 or bool((rp[1:] < rp[:-1]).any()) or int(rp[-1]) > col.numel():
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "row_ptr must start at 0, never decrease and end within col")
     if col.numel() == 0:
         col = torch.zeros(1, dtype=torch.int32, device=row_ptr.device)
     h = ctypes.c_void_p()
@@ -417,11 +456,17 @@ def lbsa_select_head_noalloc(scores, p: float, counts=None, cols=None, status=No
     Returns (counts [B*H*nB], cols [B*H*nB*nB], status [1]) int32 device
     tensors; row r's kept ids are cols[r*nB : r*nB + counts[r]].
     """
+    _on_device(scores, "scores", torch.float32)
+    if scores.dim() != 4 or scores.shape[2] != scores.shape[3]:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "scores must be [B, H, nB, nB]")
     B, H, nB, _ = scores.shape
     dev = scores.device
     counts = torch.empty(B * H * nB, dtype=torch.int32, device=dev) if counts is None else counts
     cols = torch.empty(B * H * nB * nB, dtype=torch.int32, device=dev) if cols is None else cols
     status = torch.empty(1, dtype=torch.int32, device=dev) if status is None else status
+    _on_device(counts, "counts", torch.int32, B * H * nB)
+    _on_device(cols, "cols", torch.int32, B * H * nB * nB)
+    _on_device(status, "status", torch.int32, 1)
     _check(load_library().lbsa_select_head_noalloc(_ptr(scores), B, H, nB, float(p), _ptr(counts), _ptr(cols),
                                                    _ptr(status), _stream(stream)))
     return counts, cols, status

@@ -278,7 +278,10 @@ int lbsa_blockset_export(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col
 
 /* Build a blockset from a caller CSR (device int32 row_ptr [R+1], col [nnz];
  * lists must be ascending), e.g. frozen indices saved by an earlier run.
- * Copies the data; ids are validated on the device (status word). */
+ * Copies the data; ids are validated on the device (status word).  row_ptr
+ * must be a valid CSR offset array (row_ptr[0] = 0, non-decreasing, row_ptr[R]
+ * <= the length of col): the copy reads col through it unchecked, and a row
+ * longer than nB is rejected (LBSA_ERR_BAD_INDEX, row left empty). */
 int lbsa_blockset_from_csr(const int32_t* row_ptr, const int32_t* col, int32_t B, int32_t H,
                            int32_t nB, int32_t block, lbsa_blockset** out, void* stream);
 
