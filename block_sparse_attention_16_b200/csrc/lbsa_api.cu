@@ -170,6 +170,9 @@ int scratch_alloc(DeviceState* ds, size_t bytes, cudaStream_t s, Scratch* out) {
 long long wait_limit() { return lbsa::kDefaultWaitLimit; }
 
 int new_blockset(int B, int H, int nB, int block, int scope, double p, cudaStream_t s, lbsa_blockset** out) {
+  // the kernels take the row count as an int
+  if (static_cast<long long>(B) * H * nB > 2147483647ll)
+    return fail(LBSA_ERR_UNSUPPORTED, "B*H*nB = %lld rows exceed 2^31 - 1", static_cast<long long>(B) * H * nB);
   const size_t R = static_cast<size_t>(B) * H * nB;
   const size_t cols_bytes = ((R * nB * sizeof(int32_t)) + 255) & ~size_t(255);
   const size_t counts_bytes = ((R * sizeof(int32_t)) + 255) & ~size_t(255);

@@ -162,6 +162,15 @@ def test_select_routed_rejects_bad_args():
     assert "200 KiB" in (call(H=64, nB=1024, group=64) and lbsa.lbsa_last_error())
 
 
+def test_blockset_rows_beyond_int_range_are_rejected():
+    lib = lbsa.load_library()
+    buf = np.zeros(64, dtype=np.float32)                    # host memory: rejected before any launch
+    h = ctypes.c_void_p()
+    p = ctypes.c_void_p(buf.ctypes.data)
+    assert lib.lbsa_select(p, 65535, 65535, 1, 64, 0.5, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert "2^31" in lbsa.lbsa_last_error()
+
+
 def test_call_log_reports_calls_and_errors():
     """LBSA_LOG=1: the rejected calls of a fresh process each leave a call line and an error line on stderr."""
     import subprocess
