@@ -75,7 +75,7 @@ int validate_ptr(const void* p, const char* name) {
   return LBSA_OK;
 }
 
-int n_blocks(int n_valid, int block) { return (n_valid + block - 1) / block; }
+int n_blocks(int n_valid, int block) { return static_cast<int>((static_cast<long long>(n_valid) + block - 1) / block); }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
