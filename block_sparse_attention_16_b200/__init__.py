@@ -122,8 +122,7 @@ def _ptr(t):
 def _desc(x: torch.Tensor, n_valid: int | None = None) -> _Desc:
     if x.dim() != 4 or x.stride(-1) != 1:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "expected [B, H, N, d] with a contiguous last dim")
-    if not x.is_cuda:
-        raise LbsaError(LBSA_ERR_INVALID_ARG, "tensors must live on a CUDA device")
+    _on_device(x, "q", contiguous=False)
     if x.dtype == torch.bfloat16:
         dt = 0
     elif x.dtype == torch.float32:
@@ -191,8 +190,8 @@ def lbsa_score(q, k, block: int, mode: str = "exact", scores=None, lse=None, wan
         scores = torch.empty(B, H, N if mode == "meanpool_token" else nB, nB, dtype=torch.float32, device=q.device)
     if want_lse and lse is None:
         lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device)
-    _on_device(scores, "scores", torch.float32)
-    _on_device(lse, "lse", torch.float32)
+    _on_device(scores, "scores", torch.float32, B * H * (N if mode == "meanpool_token" else nB) * nB)
+    _on_device(lse, "lse", torch.float32, B * H * N)
     _check(load_library().lbsa_score(_ptr(q), _ptr(k), ctypes.byref(desc), block, _MODES[mode],
                                      _ptr(scores), _ptr(lse), _stream(stream)))
     return (scores, lse) if (want_lse or lse is not None) else scores
@@ -423,8 +422,8 @@ def lbsa_permute(xs, perm, inverse: bool = False, outs=None, stream=None):
     for o in outs:
         _same_layout(xs[0], o)
     desc = _desc(xs[0])
-    if perm.dtype != torch.int32 or not perm.is_cuda:
-        raise LbsaError(LBSA_ERR_INVALID_ARG, "perm must be an int32 CUDA tensor")
+    # entries outside [0, N) are skipped by the kernel and reported in the device status word
+    _on_device(perm, "perm", torch.int32, xs[0].shape[2])
     n = len(xs)
     xa = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
     ya = (ctypes.c_void_p * n)(*[y.data_ptr() for y in outs])

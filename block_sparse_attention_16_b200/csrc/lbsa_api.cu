@@ -616,7 +616,10 @@ int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const in
     if ((rc = validate_ptr(ys[t], "y")) != LBSA_OK) return rc;
     if (xs[t] == ys[t]) return fail(LBSA_ERR_INVALID_ARG, "x and y may not alias");
   }
-  cudaError_t e = lbsa::launch_permute(xs, ys, count, perm, *desc, inverse, static_cast<cudaStream_t>(stream));
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != LBSA_OK) return rc;
+  cudaError_t e =
+      lbsa::launch_permute(xs, ys, count, perm, *desc, inverse, ds->status, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_permute launch");
   return LBSA_OK;
 }

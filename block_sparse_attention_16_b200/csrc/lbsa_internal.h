@@ -103,7 +103,7 @@ void partition_perm_host(int T, int Hg, int Wg, int kind, int tt, int th, int tw
 cudaError_t launch_partition_perm(int T, int Hg, int Wg, int kind, int tt, int th, int tw,
                                   int32_t* perm, cudaStream_t s);
 cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, const int32_t* perm,
-                           const lbsa_qkv_desc& d, int inverse, cudaStream_t s);
+                           const lbsa_qkv_desc& d, int inverse, int32_t* status, cudaStream_t s);
 
 cudaError_t launch_selftest_wait(long long limit_ns, int32_t* out, cudaStream_t s);
 cudaError_t launch_selftest_exp2(const float* v, float* out, long long n, cudaStream_t s);

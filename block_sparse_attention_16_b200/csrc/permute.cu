@@ -58,9 +58,11 @@ struct PtrPack {
 // CTA's iteration, 16-byte vector v) copies row slots r0 + r, r0 + r + rpi, ...
 // (32-bit row indices; every thread keeps several independent loads in flight).
 constexpr int kPermRows = 64;
+// A perm entry outside [0, N) skips its row and records LBSA_ERR_BAD_INDEX.
 __global__ void __launch_bounds__(256) permute_kernel_packed(PtrPack pk, const int32_t* __restrict__ perm, int B,
                                                              int H, int N, int vec_per_row, long long sb,
-                                                             long long sh, long long sn, int inverse) {
+                                                             long long sh, long long sn, int inverse,
+                                                             int32_t* status) {
   const int tbh = blockIdx.y;                       // tensor * (B*H) + b*H + h
   const int t = tbh / (B * H);
   const int bh = tbh - t * (B * H);
@@ -76,6 +78,10 @@ __global__ void __launch_bounds__(256) permute_kernel_packed(PtrPack pk, const i
 #pragma unroll 4
   for (int slot = r0 + lr; slot < r1; slot += rpi) {
     const int src = __ldg(perm + slot);
+    if (src < 0 || src >= N) {
+      if (v == 0) raise_status(status, LBSA_ERR_BAD_INDEX);
+      continue;
+    }
     if (!inverse) y[base + slot * sn + v] = __ldg(x + base + src * sn + v);
     else y[base + src * sn + v] = __ldg(x + base + slot * sn + v);
   }
@@ -99,7 +105,7 @@ cudaError_t launch_partition_perm(int T, int Hg, int Wg, int kind, int tt, int t
 }
 
 cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, const int32_t* perm,
-                           const lbsa_qkv_desc& d, int inverse, cudaStream_t s) {
+                           const lbsa_qkv_desc& d, int inverse, int32_t* status, cudaStream_t s) {
   const int esize = d.dtype == LBSA_BF16 ? 2 : 4;
   const int vec_per_row = d.d * esize / 16;
   const long long k = 16 / esize;   // elements per vector
@@ -114,7 +120,7 @@ cudaError_t launch_permute(const void* const* xs, void* const* ys, int count, co
   if (ybh > 65535) return cudaErrorInvalidValue;
   dim3 grid((d.N_valid + kPermRows - 1) / kPermRows, static_cast<unsigned>(ybh));
   permute_kernel_packed<<<grid, 256, 0, s>>>(pk, perm, d.B, d.H, d.N_valid, vec_per_row, d.stride_b / k, d.stride_h / k,
-                                             d.stride_n / k, inverse);
+                                             d.stride_n / k, inverse, status);
   return cudaGetLastError();
 }
 

@@ -1144,13 +1144,15 @@ extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t 
   if (!counts || !cols || !status) return set_error(LBSA_ERR_INVALID_ARG, "counts, cols and status must be non-NULL");
   if (B < 1 || H < 1 || nB < 1) return set_error(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
   if (!(p > 0.0) || !(p <= 1.0)) return set_error(LBSA_ERR_INVALID_ARG, "p must lie in (0, 1]");
+  // the same bound as lbsa_select's head scope (32-bit per-head counters need nB*nB < 2^32)
+  if (nB > 4096) return set_error(LBSA_ERR_UNSUPPORTED, "head scope is built for nB <= 4096");
   const size_t need = select_head_workspace_bytes(B, H, nB);
   if (need > kNoAllocScratchBytes) {
     char msg[200];
     std::snprintf(msg, sizeof(msg),
-                  "B*H=%d heads with nB=%d need %zu bytes of scratch; the static array holds %zu "
+                  "B*H=%lld heads with nB=%d need %zu bytes of scratch; the static array holds %zu "
                   "(B*H <= 64 with nB <= 1024 always fits)",
-                  B * H, nB, need, kNoAllocScratchBytes);
+                  static_cast<long long>(B) * H, nB, need, kNoAllocScratchBytes);
     return set_error(LBSA_ERR_UNSUPPORTED, msg);
   }
   void* ws = nullptr;

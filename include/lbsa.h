@@ -308,7 +308,10 @@ int lbsa_partition_perm(int32_t T, int32_t Hg, int32_t Wg, int32_t kind, int32_t
  *   inverse == 0:  ys[t][b,h,slot,:] = xs[t][b,h,perm[slot],:]
  *   inverse != 0:  ys[t][b,h,perm[slot],:] = xs[t][b,h,slot,:]
  * for slot < desc->N_valid; perm (device int32 [N_valid]) must be a
- * permutation of [0, N_valid).  x and y may not alias. */
+ * permutation of [0, N_valid).  An entry outside [0, N_valid) skips its row
+ * and records LBSA_ERR_BAD_INDEX in the per-device status word
+ * (lbsa_device_status); a repeated entry leaves rows unwritten (gather) or
+ * written twice (scatter).  x and y may not alias. */
 int lbsa_permute(const void* const* xs, void* const* ys, int32_t count, const int32_t* perm,
                  const lbsa_qkv_desc* desc, int32_t inverse, void* stream);
 

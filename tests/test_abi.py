@@ -197,3 +197,16 @@ def test_call_log_reports_calls_and_errors():
                            env=dict(os.environ, LBSA_LOG="0"),
                            cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=120)
     assert "[lbsa]" not in quiet.stderr
+
+
+def test_noalloc_head_selection_bounds():
+    """The allocation-free head selection takes the same nB bound as lbsa_select's
+    head scope and rejects B*H past its static scratch without overflowing the
+    head count it reports."""
+    lib = lbsa.load_library()
+    buf = np.zeros(64, dtype=np.int32)
+    p = ctypes.c_void_p(buf.ctypes.data)                    # host memory: rejected before any launch
+    assert lib.lbsa_select_head_noalloc(p, 1, 1, 4097, 0.25, p, p, p, None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert "4096" in lbsa.lbsa_last_error()
+    assert lib.lbsa_select_head_noalloc(p, 65535, 65535, 1, 0.25, p, p, p, None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert "B*H=4294836225 heads" in lbsa.lbsa_last_error()
