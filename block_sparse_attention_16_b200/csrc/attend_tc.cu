@@ -42,6 +42,13 @@ constexpr int kThreads = 192;
 constexpr int kMaxBlocks = 4096;  // nB bound (bitmap size)
 constexpr int kMaxWords = kMaxBlocks / 32;
 constexpr uint32_t kTmemCols = 256;
+// kPoly8 of every 8 pairs of logits of a step without masked keys take their
+// exponentials on the FMA pipe (scalar cubic, relative error < 8e-5, far below
+// bf16's rounding of P), which unloads the MUFU; 0 keeps every one on the MUFU
+#ifndef LBSA_ATT_POLY8
+#define LBSA_ATT_POLY8 0
+#endif
+constexpr int kPoly8 = LBSA_ATT_POLY8;
 template <int D>
 struct Layout {
   static constexpr int Q_BYTES = BM * D * 2;
@@ -422,7 +429,8 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         for (int c = 0; c < 32; ++c) {
           float v0, v1;
           u64_as_f2(ffma2(f2_as_u64(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])), sc2, nm2), v0, v1);
-          const float p0 = ex2(v0), p1 = ex2(v1);
+          const bool poly = ((c * kPoly8) & 7) < kPoly8;
+          const float p0 = poly ? exp2_poly3(v0) : ex2(v0), p1 = poly ? exp2_poly3(v1) : ex2(v1);
           sum4[c & 3] = fadd2(sum4[c & 3], f2_as_u64(p0, p1));
           pk[c] = pack_bf16x2(p0, p1);
         }

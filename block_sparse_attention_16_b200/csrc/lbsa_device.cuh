@@ -113,6 +113,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// One lane of the (fully active) warp returns true.  A warp that walks a loop
+// together keeps its loop values warp-uniform, and the elected lane issues the
+// single-thread instructions (UMMA, commit) with them.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r));
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 // 4D tiled load (coords innermost first) into shared memory, completing
 // `bytes` on `bar`.  The x coordinate is always a multiple of 64 elements.
@@ -203,6 +216,27 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The same wait, with the 32 registers of one earlier tmem_ld32 as operands: no
+// use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+// Orders later uses of 32 registers after the preceding (volatile) wait.
+__device__ __forceinline__ void reg_dep(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------------ descriptors
@@ -280,6 +314,23 @@ __device__ __forceinline__ unsigned long long exp2_poly2(unsigned long long v2) 
   const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
   return (static_cast<unsigned long long>(hi) << 32) | lo;
 }
+// 2^v for v <= 8 on the FMA pipe (no MUFU), scalar: the same round-to-nearest
+// range reduction as exp2_poly2, then a cubic fitted the same way (minimax
+// relative error on [-1/2, 1/2] by iteratively reweighted least squares on
+// Chebyshev nodes: 7.5e-5 with the fp32-rounded coefficients), for softmax
+// probabilities that are rounded to bf16 (relative rounding 2^-9) afterwards.
+// Scalar because packed fp32x2 operations take the FMA pipe as long as two
+// scalar ones.  Inputs below -125 are clamped there.
+__device__ __forceinline__ float exp2_poly3(float v) {
+  v = fmaxf(v, -125.f);
+  const float t = v + 12582912.f;                        // low bits: rint(v)
+  const float f = v - (t - 12582912.f);                  // in [-1/2, 1/2]
+  float q = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  q = fmaf(q, f, 0.6932609677314758f);
+  q = fmaf(q, f, 0.9999280571937561f);
+  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

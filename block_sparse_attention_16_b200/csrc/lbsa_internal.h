@@ -56,6 +56,12 @@ struct ScoreArgs {
 // bf16 tcgen05 kernels (attend_tc.cu, score_tc.cu)
 cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                                const AttendArgs& a, cudaStream_t s);
+// two query tiles per CTA in ping-pong, 128-key steps (attend_pp.cu): any blockset
+// without per-token masks (lbsa_attend gives it the dense ones); the Q map's box is
+// 128 rows, the K and V maps' 64 rows
+bool attend_pp_supported(const AttendArgs& a);
+cudaError_t launch_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                  const AttendArgs& a, cudaStream_t s);
 // dense attention that also writes the exact block masses (a.scores); a.counts/cols unused
 cudaError_t launch_score_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                                      const AttendArgs& a, cudaStream_t s);
