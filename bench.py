@@ -1,21 +1,33 @@
-"""Benchmark of the block-sparse video-attention hot path on B200.
+"""Benchmark of block-sparse video attention on B200.
 
-One step = one pass of the whole path over one Wan-like attention layer
-(B=1, H=12, d=128, 21x30x52 = 32,760 tokens, bf16, 64-token blocks):
-  3D-tile permutation of Q, K, V  ->  exact block mass (two-sweep dense pass)
-  ->  fixed-point row selection at p = 0.99  ->  block-sparse attention
-  ->  inverse permutation of O.
-Inputs are resident in HBM when timing starts (302 MB of Q/K/V per step, larger
-than the 126 MB L2, so no extra flush is needed between steps).
+One step = one block-sparse attention call over one Wan-like attention layer
+(B=1, H=12, d=128, 21x30x52 = 32,760 tokens in 3D-tile order, bf16, 64-token
+blocks) with block indices selected once at p = 0.99 from exact block masses
+and then frozen: LoSA's steady state, and the metric's own quantity.  Inputs
+are resident in HBM when timing starts (302 MB of Q/K/V, larger than the
+126 MB L2, so no extra flush is needed between calls).
 
-value  = algorithmic TFLOP/s of the whole step, summed over ranks:
-         exact mass 2*N^2*d*H (one Q K^T) + attention 4*d*sum_kept(valid_q*valid_k)
-         per step, divided by the max-over-ranks device time of the K steps.
+value  = TFLOP/s on the kept pairs, summed over ranks: 4*d*sum_kept(valid_q *
+         valid_k) per call, divided by the max-over-ranks device time per call.
+The same JSON line carries, measured in the same run (single GPU):
+  attend    ms/call, TFLOP/s and fraction of the measured burst bf16 peak
+  dense     our kernel at p = 1 and torch SDPA on the same layer
+  step0     LoSA's one dense step: fused dense attention + exact masses, then
+            selection; and the exact scorer alone
+  hot_path  one pass of the whole path: permute, exact masses, selection,
+            attention, inverse permute
+  config2   HunyuanVideo-like layer: indices from step 0, then 49 re-drawn
+            attention calls with them frozen (median, p10, p90 per call)
+  config4   skewed heads, p in {0.90, 0.95, 0.99, 0.999}: ms, TFLOP/s, density
+  config3   mean-pooled proxy with head-scope tau = 0.25, per partition (1D,
+            2D, 3D): the whole call
+  config0   the tiny fp32 case: scorer, selection, attention
 Multi-GPU (--gpus N under torchrun): every rank runs its own layer (the path
 shards by (batch, head) with no exchange step), so scaling is weak and there is
 no data-path collective.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+                  [--no-extra] [--clocks-csv PATH]
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
 build) on a bounded sample of the same workload on the host cores.
@@ -159,8 +171,9 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- oracle (CPU) sample
-def oracle_sample(q, k, v, wl, heads_qblocks, p=P):
-    """Run the fp64 oracle on sampled (head, query block) units; returns (flops, seconds)."""
+def oracle_attention_sample(q, k, v, wl, row_ptr, col, heads_qblocks):
+    """The fp64 oracle's block-sparse attention on sampled (head, query block)
+    units of a blockset (CSR over B*H*nB rows); returns (kept-pair FLOPs, seconds)."""
     import oracle
     nB, b, n, d = wl.n_blocks, wl.block, wl.n_valid, wl.d
     flops = 0.0
@@ -169,23 +182,29 @@ def oracle_sample(q, k, v, wl, heads_qblocks, p=P):
         qh = q[:, h:h + 1].float().numpy()
         kh = k[:, h:h + 1].float().numpy()
         vh = v[:, h:h + 1].float().numpy()
-        mass = oracle.block_mass(qh, kh, n, b, qblocks=qbs)
-        rows = []
-        for t, i in enumerate(qbs):
-            seg = mass[:, :, t:t + 1, :].astype(np.float32)
-            rp, col = oracle.select_contract(seg, p, "row")
-            rows.append(col)
-        full = [np.zeros(0, dtype=np.int64)] * nB
-        for i, c in zip(qbs, rows):
-            full[i] = c
-        rp, col = oracle.csr_from_rows(full)
-        oracle.sparse_attention(qh, kh, vh, n, b, rp, col, qblocks=qbs)
-        for i, c in zip(qbs, rows):
+        rp = row_ptr[h * nB:(h + 1) * nB + 1] - row_ptr[h * nB]
+        cl = col[row_ptr[h * nB]:row_ptr[(h + 1) * nB]]
+        oracle.sparse_attention(qh, kh, vh, n, b, rp, cl, qblocks=qbs)
+        for i in qbs:
             vq = min(b, n - i * b)
-            flops += 2.0 * vq * n * d
-            vk = sum(min(b, n - j * b) for j in c)
+            vk = sum(min(b, n - j * b) for j in cl[rp[i]:rp[i + 1]])
             flops += 4.0 * d * vq * vk
     return flops, time.perf_counter() - t0
+
+
+def oracle_frozen_rows(q, k, wl, heads_qblocks, p=P):
+    """Step 0 on the host: exact masses of the sampled query blocks and the
+    fixed-point selection (the untimed set-up of the reference arm); returns a
+    CSR over all B*H*nB rows whose other rows are empty."""
+    import oracle
+    nB, b, n = wl.n_blocks, wl.block, wl.n_valid
+    rows = [np.zeros(0, dtype=np.int64)] * (wl.H * nB)
+    for h, qbs in heads_qblocks:
+        mass = oracle.block_mass(q[:, h:h + 1].float().numpy(), k[:, h:h + 1].float().numpy(), n, b, qblocks=qbs)
+        for t, i in enumerate(qbs):
+            _, c = oracle.select_contract(mass[:, :, t:t + 1, :].astype(np.float32), p, "row")
+            rows[h * nB + i] = c
+    return oracle.csr_from_rows(rows)
 
 
 def cores():
@@ -212,11 +231,15 @@ def run_reference(args, rank, world):
         h = step % wl.H
         return [(h, sorted(rng.choice(wl.n_blocks, per_step, replace=False).tolist()))]
 
+    samples = [sample(s) for s in range(args.warmup + args.steps)]
+    # set-up (untimed, as the frozen indices are for the GPU arm): step 0's masses
+    # and selection for every sampled query block
+    rp, col = oracle_frozen_rows(q, k, wl, [u for smp in samples for u in smp])
     for s in range(args.warmup):
-        oracle_sample(q, k, v, wl, sample(s))
+        oracle_attention_sample(q, k, v, wl, rp, col, samples[s])
     tot_f, tot_t = 0.0, 0.0
     for s in range(args.steps):
-        f, t = oracle_sample(q, k, v, wl, sample(args.warmup + s))
+        f, t = oracle_attention_sample(q, k, v, wl, rp, col, samples[args.warmup + s])
         tot_f += f
         tot_t += t
     value = tot_f / tot_t / 1e12
@@ -227,8 +250,9 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(wl, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": n_cores, "kind": "oracle",
-                         "sample": f"{per_step} query blocks of one head per step (exact mass row sweep, "
-                                   f"fixed-point selection, sparse attention) on the 3D-tile-ordered layer"},
+                         "sample": f"block-sparse attention of {per_step} query blocks of one head per step, "
+                                   f"indices from the oracle's exact masses and p = {P} selection (untimed set-up), "
+                                   f"3D-tile-ordered Wan-like layer"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -238,13 +262,148 @@ def run_reference(args, rank, world):
 def config_dict(wl, world):
     T, H, W = wl.grid
     return {"workload": f"Wan-like layer {T}x{H}x{W} ({wl.n_valid} tokens), H={wl.H}, d={wl.d}, "
-                        f"{wl.block}-token blocks, 3D 4x4x4 tiles, exact mass, p={P}",
+                        f"{wl.block}-token blocks, 3D 4x4x4 tiles: one block-sparse attention call with "
+                        f"indices selected at p={P} from exact block masses and frozen",
             "B": wl.B, "H": wl.H, "d": wl.d, "n_valid": wl.n_valid, "block": wl.block, "p": P,
-            "partition": "3d tiles 4x4x4", "l2": "inputs larger than L2 (302 MB Q/K/V per step)",
+            "partition": "3d tiles 4x4x4", "l2": "inputs larger than L2 (302 MB Q/K/V per call)",
             "parallelism": f"replicas x{world} (independent layers, no collective)"}
 
 
 # ---------------------------------------------------------------- own arm
+def blockset_flops(lbsa, bs, wl):
+    """Kept-pair attention FLOPs and density of a row- or head-scope blockset."""
+    rp, col = lbsa.lbsa_blockset_export(bs)
+    rp, col = rp.cpu().numpy(), col.cpu().numpy()
+    R = wl.B * wl.H * wl.n_blocks
+    mask = kept_mask(rp, col, R, wl.n_blocks).reshape(wl.B * wl.H, wl.n_blocks, wl.n_blocks)
+    return attention_flops(mask, wl.n_blocks, wl.block, wl.n_valid, wl.d), float(mask.mean()), rp, col
+
+
+def dense_flops(wl):
+    return 4.0 * wl.d * wl.n_valid ** 2 * wl.H * wl.B
+
+
+def extra_measurements(lbsa, wl, dev, qp, kp, vp, perm, q, k, v, pk):
+    """Everything the line reports beside the contract's timed calls (single GPU)."""
+    from block_sparse_attention_16_b200.workload import get_workload, make_qkv, make_qkv_f32, redraw_qkv
+
+    def tf(fl, ms):
+        return fl / (ms * 1e-3) / 1e12
+
+    out = {}
+    # dense attention on the same layer: our kernel at p = 1 (every block) and torch SDPA
+    nB = wl.n_blocks
+    full = torch.full((wl.B, wl.H, nB, nB), 1.0 / nB, device=dev)
+    bs1 = lbsa.lbsa_select(full, wl.block, 1.0, "row")
+    fd = dense_flops(wl)
+    t_own = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs1))["median"]
+    t_sdpa = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp))["median"]
+    out["dense"] = {"own_p1_ms": t_own, "own_p1_tflops": tf(fd, t_own), "torch_sdpa_ms": t_sdpa,
+                    "torch_sdpa_tflops": tf(fd, t_sdpa), "flops": fd}
+    # LoSA's one dense step: fused dense attention + exact masses, then selection
+    sc_f, o_f = lbsa.lbsa_score_attend(qp, kp, vp, wl.block)
+    t_fused = _timer(lambda: lbsa.lbsa_score_attend(qp, kp, vp, wl.block, scores=sc_f, out=o_f))["median"]
+    t_sel = _timer(lambda: lbsa.lbsa_select(sc_f, wl.block, P, "row"))["median"]
+    sc = lbsa.lbsa_score(qp, kp, wl.block)
+    t_score = _timer(lambda: lbsa.lbsa_score(qp, kp, wl.block, scores=sc))["median"]
+    out["step0"] = {"fused_dense_step_ms": t_fused, "select_ms": t_sel, "total_ms": t_fused + t_sel,
+                    "fused_vs_own_dense": t_fused / t_own, "exact_scorer_ms": t_score,
+                    "exact_scorer_tflops": tf(2.0 * wl.n_valid ** 2 * wl.d * wl.H, t_score)}
+
+    # one pass of the whole path
+    def hot():
+        a_, b_, c_ = lbsa.lbsa_permute([q, k, v], perm)
+        s_ = lbsa.lbsa_score(a_, b_, wl.block)
+        x_ = lbsa.lbsa_select(s_, wl.block, P, "row")
+        o_ = lbsa.lbsa_attend(a_, b_, c_, x_)
+        return lbsa.lbsa_permute([o_], perm, inverse=True)[0]
+    out["hot_path"] = {"ms": _timer(hot)["median"],
+                       "stages": "3D permute of Q, K, V; exact masses; row selection p=0.99; attention; "
+                                 "inverse permute of O"}
+
+    # config 2: HunyuanVideo-like layer, indices from step 0, 49 re-drawn calls with them frozen
+    wh = get_workload("hunyuan")
+    q32, k32, v32 = make_qkv_f32(wh, device=dev)
+    qh, kh, vh = (x.to(torch.bfloat16) for x in (q32, k32, v32))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    sch, _ = lbsa.lbsa_score_attend(qh, kh, vh, wh.block)
+    bsh = lbsa.lbsa_select(sch, wh.block, P, "row")
+    e1.record()
+    torch.cuda.synchronize()
+    t_step0 = e0.elapsed_time(e1)
+    flh, densh, _, _ = blockset_flops(lbsa, bsh, wh)
+    calls = []
+    for t in range(1, wh.extra["steps"] + 1):
+        qh, kh, vh = redraw_qkv(wh, q32, k32, v32, t)
+        e0.record()
+        lbsa.lbsa_attend(qh, kh, vh, bsh)
+        e1.record()
+        e1.synchronize()
+        calls.append(e0.elapsed_time(e1))
+    calls.sort()
+    med = calls[len(calls) // 2]
+    t_sdpa_h = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qh, kh, vh), n=3, warm=1)["median"]
+    out["config2"] = {"workload": "HunyuanVideo-like 33x45x80 (118800 tokens), H=24, d=128, 128-token blocks, raster",
+                      "step0_ms": t_step0, "calls": len(calls), "density": densh, "ms_per_call_median": med,
+                      "ms_per_call_p10": calls[max(0, len(calls) // 10)],
+                      "ms_per_call_p90": calls[min(len(calls) - 1, 9 * len(calls) // 10)],
+                      "tflops_median": tf(flh, med), "frac_of_burst": tf(flh, med) / pk["bf16"],
+                      "torch_sdpa_dense_ms": t_sdpa_h, "torch_sdpa_dense_tflops": tf(dense_flops(wh), t_sdpa_h)}
+    assert lbsa.lbsa_get_status(bsh) == 0
+    del q32, k32, v32, qh, kh, vh, sch, bsh
+
+    # config 4: skewed heads, p sweep
+    ws = get_workload("wan_skew")
+    T, H, W = ws.grid
+    qs, ks, vs = make_qkv(ws, device=dev)
+    perm_s = lbsa.lbsa_partition_perm(T, H, W, "3d", device=dev)
+    qs, ks, vs = lbsa.lbsa_permute([qs, ks, vs], perm_s)
+    scs = lbsa.lbsa_score(qs, ks, ws.block)
+    rows = []
+    for p_ in ws.extra["p_sweep"]:
+        bsp = lbsa.lbsa_select(scs, ws.block, p_, "row")
+        fl, dens, _, _ = blockset_flops(lbsa, bsp, ws)
+        ta = _timer(lambda: lbsa.lbsa_attend(qs, ks, vs, bsp))["median"]
+        rows.append({"p": p_, "density": dens, "attend_ms": ta, "tflops": tf(fl, ta), "frac_of_burst": tf(fl, ta) / pk["bf16"]})
+    t_d = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qs, ks, vs))["median"]
+    out["config4"] = {"workload": "skewed heads (half alpha in [2,4], half in [0.25,0.5]), Wan-like shape",
+                      "rows": rows, "torch_sdpa_dense_ms": t_d}
+    del qs, ks, vs, scs
+
+    # config 3: mean-pooled proxy, head scope tau = 0.25, one whole call per partition
+    wp = get_workload("wan_proxy")
+    T, H, W = wp.grid
+    qq, kk, vv = make_qkv(wp, device=dev)
+    prow = {}
+    for part in ("1d", "2d", "3d"):
+        pm = lbsa.lbsa_partition_perm(T, H, W, part, device=dev)
+
+        def call():
+            a_, b_, c_ = lbsa.lbsa_permute([qq, kk, vv], pm)
+            s_ = lbsa.lbsa_score(a_, b_, wp.block, mode="meanpool")
+            x_ = lbsa.lbsa_select(s_, wp.block, wp.p, "head")
+            o_ = lbsa.lbsa_attend(a_, b_, c_, x_)
+            return lbsa.lbsa_permute([o_], pm, inverse=True)[0]
+        prow[part] = _timer(call)["median"]
+    out["config3"] = {"workload": "mean-pooled proxy, head scope tau=0.25, Wan-like shape",
+                      "call_ms": prow, "call_ms_mean_of_cycle": sum(prow.values()) / 3}
+    del qq, kk, vv
+
+    # config 0: tiny fp32 case
+    wt = get_workload("tiny")
+    qt, kt, vt = (x.to(dev) for x in make_qkv(wt))
+    sct = lbsa.lbsa_score(qt, kt, wt.block)
+    bst = lbsa.lbsa_select(sct, wt.block, P, "row")
+    out["config0"] = {"workload": "tiny fp32 (2 heads, 256 tokens, d=64)",
+                      "score_ms": _timer(lambda: lbsa.lbsa_score(qt, kt, wt.block, scores=sct))["median"],
+                      "select_ms": _timer(lambda: lbsa.lbsa_select(sct, wt.block, P, "row"))["median"],
+                      "attend_ms": _timer(lambda: lbsa.lbsa_attend(qt, kt, vt, bst))["median"]}
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_device_status() == 0
+    return out
+
+
 def run_own(args, rank, world):
     import block_sparse_attention_16_b200 as lbsa
     from block_sparse_attention_16_b200.build import build
@@ -262,85 +421,54 @@ def run_own(args, rank, world):
     q, k, v = make_qkv(wl, device=dev)
     perm = lbsa.lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4), device=dev)
     stream = torch.cuda.current_stream()
-    nB = wl.n_blocks
 
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
-        if ev:
-            ev[1].record(stream)
-        scores = lbsa.lbsa_score(qp, kp, wl.block)
-        if ev:
-            ev[2].record(stream)
-        bs = lbsa.lbsa_select(scores, wl.block, P, "row")
-        if ev:
-            ev[3].record(stream)
-        op = lbsa.lbsa_attend(qp, kp, vp, bs)
-        if ev:
-            ev[4].record(stream)
-        o = lbsa.lbsa_permute([op], perm, inverse=True)[0]
-        if ev:
-            ev[5].record(stream)
-        return o, bs
+    # step 0 (untimed): 3D-tile order, exact masses, selection at p = 0.99; the
+    # indices are then frozen for every timed call (LoSA's schedule)
+    qp, kp, vp = lbsa.lbsa_permute([q, k, v], perm)
+    scores = lbsa.lbsa_score(qp, kp, wl.block)
+    bs = lbsa.lbsa_select(scores, wl.block, P, "row")
+    att_flops, density, rp, col = blockset_flops(lbsa, bs, wl)
+    out = torch.empty_like(qp)
 
     for _ in range(args.warmup):
-        o, bs = step()
+        lbsa.lbsa_attend(qp, kp, vp, bs, out=out)
     torch.cuda.synchronize()
-    rp, col = lbsa.lbsa_blockset_export(bs)
-    rp, col = rp.cpu().numpy(), col.cpu().numpy()
-    R = wl.B * wl.H * nB
-    mask = kept_mask(rp, col, R, nB).reshape(wl.B * wl.H, nB, nB)
-    att_flops = attention_flops(mask, nB, wl.block, wl.n_valid, wl.d)
-    score_flops = 2.0 * wl.n_valid ** 2 * wl.d * wl.H * wl.B
-    step_flops = att_flops + score_flops
-    density = float(mask.mean())
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    clocks = Clocks(dev.index, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-                    if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/lbsa_clocks_{rank}.csv")
+    clocks_path = args.clocks_csv or f"/tmp/lbsa_clocks_rank{rank}.csv"
+    clocks = Clocks(dev.index, clocks_path)
     barrier(dev)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for s in range(args.steps):
-        o, bs = step(evs[s])
+    for _ in range(args.steps):
+        lbsa.lbsa_attend(qp, kp, vp, bs, out=out)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(dev)
     clk = clocks.stop()
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
-    stage_names = ["permute", "score", "select", "attend", "unpermute"]
-    stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, n in enumerate(stage_names)}
     ms_per_step = total_ms / args.steps
-    value = world * step_flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = world * att_flops * args.steps / (total_ms * 1e-3) / 1e12
+    assert lbsa.lbsa_get_status(bs) == 0
 
     pk = peaks()
-    att_ms = stages["attend"]
-    sc_ms = stages["score"]
-    att_tflops = att_flops / (att_ms * 1e-3) / 1e12
-    sc_tflops = score_flops / (sc_ms * 1e-3) / 1e12
-    dominant = "attend" if att_ms >= sc_ms else "score"
-    dom_flops = att_flops if dominant == "attend" else score_flops
-    dom_ms = max(att_ms, sc_ms)
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    traffic = load_traffic(dominant)
-    roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": pk["bf16_sustained"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"], "traffic": traffic,
-                "peak_source": pk["source"] + " (bf16 sustained; kernel timed inside a step)"}
+    att_tflops = att_flops / (ms_per_step * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attend", "achieved": att_tflops, "peak": pk["bf16"],
+                "unit": "TFLOP/s", "frac": att_tflops / pk["bf16"], "traffic": load_traffic("attend"),
+                "peak_source": pk["source"] + " (bf16 burst: the attention call is the whole timed step)"}
 
-    # end to end through the public API: every step uploads its Q, K, V from
-    # pinned host memory, runs the path and downloads its output.  Two steps are
-    # in flight: step i+1's inputs upload (copy stream) while step i computes,
-    # and step i's output downloads (second copy stream) while step i+1 computes.
-    qh, kh, vh = (x.cpu().pin_memory() for x in (q, k, v))
+    # end to end through the public API: every step uploads its Q, K, V (block
+    # order) from pinned host memory, runs the attention call with the frozen
+    # indices and downloads O.  Two steps are in flight: step i+1's inputs upload
+    # (copy stream) while step i computes, and step i's output downloads (second
+    # copy stream) while step i+1 computes.
+    qh, kh, vh = (x.cpu().pin_memory() for x in (qp, kp, vp))
     ohs = [torch.empty_like(qh).pin_memory() for _ in range(2)]
-    ins = [[torch.empty_like(q) for _ in range(3)] for _ in range(2)]
-    outs = [torch.empty_like(q) for _ in range(2)]
+    ins = [[torch.empty_like(qp) for _ in range(3)] for _ in range(2)]
+    outs = [torch.empty_like(qp) for _ in range(2)]
     h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]      # slot's inputs have landed
-    ev_free = [torch.cuda.Event() for _ in range(2)]    # slot's inputs consumed (permuted)
+    ev_free = [torch.cuda.Event() for _ in range(2)]    # slot's inputs consumed
     ev_out = [torch.cuda.Event() for _ in range(2)]     # slot's output ready on the device
     ev_down = [torch.cuda.Event() for _ in range(2)]    # slot's output downloaded
     started = [False, False]
@@ -357,21 +485,16 @@ def run_own(args, rank, world):
     def compute(i):
         sl = i % 2
         stream.wait_event(ev_in[sl])
-        qp, kp, vp = lbsa.lbsa_permute(ins[sl], perm)
-        ev_free[sl].record(stream)
-        scores = lbsa.lbsa_score(qp, kp, wl.block)
-        bsx = lbsa.lbsa_select(scores, wl.block, P, "row")
-        op = lbsa.lbsa_attend(qp, kp, vp, bsx)
         if started[sl]:
             stream.wait_event(ev_down[sl])
-        lbsa.lbsa_permute([op], perm, inverse=True, outs=[outs[sl]])
+        lbsa.lbsa_attend(*ins[sl], bs, out=outs[sl])
+        ev_free[sl].record(stream)
         ev_out[sl].record(stream)
         d2h.wait_event(ev_out[sl])
         with torch.cuda.stream(d2h):
             ohs[sl].copy_(outs[sl], non_blocking=True)
         ev_down[sl].record(d2h)
         started[sl] = True
-        return bsx
 
     def e2e_run(n, e_begin=None):
         if e_begin is not None:
@@ -393,35 +516,40 @@ def run_own(args, rank, world):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     bytes_in = 3 * q.numel() * q.element_size()
     bytes_out = q.numel() * q.element_size()
+    del qh, kh, vh, ohs, ins, outs
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        qc, kc, vc = (x[:, :, perm.long()].cpu() for x in (q, k, v))
+        qc, kc, vc = (x.cpu() for x in (qp, kp, vp))
         rng = np.random.default_rng(1)
-        sample = [(h, sorted(rng.choice(nB, 4, replace=False).tolist())) for h in range(0, wl.H, 2)]
-        f, t = oracle_sample(qc, kc, vc, wl, sample)
+        sample = [(h, sorted(rng.choice(wl.n_blocks, 4, replace=False).tolist())) for h in range(0, wl.H, 2)]
+        f, t = oracle_attention_sample(qc, kc, vc, wl, rp.astype(np.int64), col.astype(np.int64), sample)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": cores(), "kind": "oracle",
-               "sample": f"{sum(len(x[1]) for x in sample)} query blocks over {len(sample)} heads "
-                         f"(exact mass row sweep, fixed-point selection, sparse attention), {t:.1f} s"}
+               "sample": f"block-sparse attention of {sum(len(x[1]) for x in sample)} query blocks over "
+                         f"{len(sample)} heads with the frozen indices, {t:.1f} s"}
+
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra = extra_measurements(lbsa, wl, dev, qp, kp, vp, perm, q, k, v, pk)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl, world),
-            "stages_ms": stages, "density": density,
-            "attend": {"ms_per_call": att_ms, "tflops": att_tflops,
-                       "frac": att_tflops / pk["bf16_sustained"], "flops_per_call": att_flops},
-            "score": {"ms_per_call": sc_ms, "tflops": sc_tflops, "flops_per_call": score_flops},
+            "attend": {"ms_per_call": ms_per_step, "tflops": att_tflops, "frac_of_burst": att_tflops / pk["bf16"],
+                       "flops_per_call": att_flops, "density": density},
             "roofline": roofline,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * step_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": world * att_flops * args.steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "ms_per_step": e2e_ms / args.steps,
                     "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": bytes_out,
                     "overlap": "two steps in flight: uploads and downloads on two copy streams"},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": args.steps,
             "clocks": clk,
         }
+        if extra:
+            line.update(extra)
         print(json.dumps(line), flush=True)
     return 0
 
@@ -739,10 +867,13 @@ def run_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="leave out the measurements beside the contract's timed calls (dense, step 0, configs 0-4)")
+    ap.add_argument("--clocks-csv", default=None, help="where the nvidia-smi clock samples go (default under /tmp)")
     ap.add_argument("--profile", choices=["attend", "score", "select", "proxy", "token", "routed"],
                     help="run the small ncu case for one kernel instead of the benchmark")
     ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
