@@ -312,7 +312,6 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
   if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
   if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
   if (scope != LBSA_SCOPE_ROW && scope != LBSA_SCOPE_HEAD) return fail(LBSA_ERR_INVALID_ARG, "scope %d", scope);
-  if (scope == LBSA_SCOPE_ROW && nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "row scope is built for nB <= 1024");
   if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "nB %d > 4096", nB);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   lbsa_blockset* bs = nullptr;
@@ -348,7 +347,7 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
   if ((rc = validate_ptr(scores, "scores")) != LBSA_OK) return rc;
   if (B < 1 || H < 1 || nB < 1) return fail(LBSA_ERR_INVALID_ARG, "B, H, nB must be >= 1");
   if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
-  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "the rank rules are built for nB <= 1024");
+  if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "the rank rules are built for nB <= 4096");
   if (static_cast<long long>(nB - 1) * block >= n_valid || n_valid > static_cast<long long>(nB) * block)
     return fail(LBSA_ERR_INVALID_ARG, "n_valid %d does not match nB %d x block %d", n_valid, nB, block);
   if (rule == LBSA_RULE_LOCAL_TOPK) {
@@ -398,7 +397,7 @@ int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_vali
   if (block != 64) return fail(LBSA_ERR_UNSUPPORTED, "per-token scope is built for 64-token blocks (block %d)", block);
   if (!(p > 0.0) || !(p <= 1.0) || std::isnan(p)) return fail(LBSA_ERR_INVALID_ARG, "p = %g not in (0, 1]", p);
   const int nB = n_blocks(n_valid, block);
-  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "per-token scope is built for nB <= 1024 (nB %d)", nB);
+  if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "per-token scope is built for nB <= 4096 (nB %d)", nB);
   if (static_cast<long long>(n_valid) * nB > 65535ll * 4096)
     return fail(LBSA_ERR_UNSUPPORTED, "%d tokens x %d blocks per head exceed the histogram grid", n_valid, nB);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -435,7 +434,7 @@ int lbsa_select_routed(const float* scores, int32_t B, int32_t H, int32_t nB, in
   if (std::isnan(entropy_threshold)) return fail(LBSA_ERR_INVALID_ARG, "entropy threshold is NaN");
   if (group < 1) return fail(LBSA_ERR_INVALID_ARG, "group = %d < 1", group);
   if (H > 4096) return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for H <= 4096 (H %d)", H);
-  if (nB > 1024) return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for nB <= 1024 (nB %d)", nB);
+  if (nB > 4096) return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for nB <= 4096 (nB %d)", nB);
   if (static_cast<long long>(B) * H > 65535)
     return fail(LBSA_ERR_UNSUPPORTED, "routed scope is built for B*H <= 65535 heads (%d x %d)", B, H);
   const size_t smem = lbsa::select_routed_smem_bytes(H, nB, group);

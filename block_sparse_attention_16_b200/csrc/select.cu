@@ -142,6 +142,153 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
   if (lane == 0) counts[row] = base;
 }
 
+// ---------------------------------------------------------------- wide rows
+// Rows of more than 1024 blocks (up to 4096): one 256-thread CTA per row,
+// thread t holding elements t, t + 256, ...; the same threshold search as the
+// one-warp kernels above with CTA-wide exact sums, then an ascending emit by
+// CTA-wide prefix counts.  kind 0: the threshold rule on fixed-point weights
+// (skip_head as in select_row_kernel); kind 1: the row's own block plus the k
+// top-ranked others (Local + TopK); kind 2: the first max(c, min(K, nB)) of the
+// ranked order (per-head floor), rows with n == c left as they are.
+constexpr int kWideThreads = 256;
+
+// Exact CTA sum of per-thread values below 2^54 (< 2^62 in total); buf is one
+// of two [8] slots used alternately, so one barrier per call suffices.
+__device__ __forceinline__ uint64_t cta_sum_u64(uint64_t v, unsigned long long* buf) {
+  v = warp_sum_u64(v);
+  if ((threadIdx.x & 31) == 0) buf[threadIdx.x >> 5] = v;
+  __syncthreads();
+  uint64_t t = 0;
+#pragma unroll
+  for (int w = 0; w < kWideThreads / 32; ++w) t += buf[w];
+  return t;
+}
+
+// Exclusive CTA prefix count of a per-thread flag in thread order, and the total.
+__device__ __forceinline__ uint32_t cta_prefix(bool f, uint32_t* buf, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t m = __ballot_sync(0xffffffffu, f);
+  if (lane == 0) buf[warp] = __popc(m);
+  __syncthreads();
+  uint32_t before = 0;
+  total = 0;
+#pragma unroll
+  for (int w = 0; w < kWideThreads / 32; ++w) {
+    const uint32_t c = buf[w];
+    before += (w < warp) ? c : 0u;
+    total += c;
+  }
+  return before + __popc(m & ((1u << lane) - 1u));
+}
+
+template <int EPT>
+__global__ void __launch_bounds__(kWideThreads) select_wide_kernel(
+    const float* __restrict__ scores, int R, int nB, int kind, uint32_t Pfix, int keep_all, int k,
+    const int32_t* __restrict__ head_floor, int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+    int32_t* __restrict__ status, const int32_t* __restrict__ skip_head) {
+  __shared__ unsigned long long red[2][kWideThreads / 32];
+  __shared__ uint32_t cnt[4][kWideThreads / 32];
+  const long long row = blockIdx.x;
+  if (row >= R) return;                                     // CTA-uniform
+  if (kind == 0 && skip_head && skip_head[row / nB] >= 0) return;
+  const int t = threadIdx.x;
+  const int diag = (kind == 1) ? static_cast<int>(row % nB) : -1;
+  int n = 0;
+  if (kind == 1) {
+    n = min(k, nB - 1);
+  } else if (kind == 2) {
+    const int c = counts[row];
+    n = max(c, min(head_floor[row / nB], nB));
+    if (n == c) return;
+  }
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
+  int32_t* out = cols + row * nB;
+  uint32_t bits[EPT];
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const int idx = e * kWideThreads + t;
+    bits[e] = (idx < nB) ? __ldg(x + idx) : 0u;
+    bad |= (idx < nB) && (bits[e] >= kInvalidBits);
+  }
+  int step = 0;                                             // alternates the two reduction slots
+  if (__syncthreads_or(bad)) {
+    if (t == 0) raise_status(status, LBSA_ERR_INVALID_SCORES);
+    for (int idx = t; idx < nB; idx += kWideThreads) out[idx] = idx;
+    if (t == 0) counts[row] = nB;
+    return;
+  }
+  if (kind == 0 && keep_all) {
+    for (int idx = t; idx < nB; idx += kWideThreads) out[idx] = idx;
+    if (t == 0) counts[row] = nB;
+    return;
+  }
+  // weight of element e: its fixed-point mass (kind 0) or 1 (ranked kinds)
+  auto weight = [&](int e) -> uint64_t {
+    const int idx = e * kWideThreads + t;
+    if (idx >= nB || idx == diag) return 0;
+    return kind == 0 ? fixed_weight(bits[e]) : 1ull;
+  };
+  uint64_t T;
+  if (kind == 0) {
+    uint64_t ws = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) ws += weight(e);
+    T = threshold_T(cta_sum_u64(ws, red[step++ & 1]), Pfix);
+  } else {
+    T = static_cast<uint64_t>(n);
+  }
+  uint32_t tb = 0u, need = 0u;
+  bool none = kind != 0 && n == 0;                          // ranked kinds with nothing ranked in
+  if (!none && T == 0) {
+    // nothing to reach (kind 0): keep one block, the highest score with the lowest index
+    uint32_t mb = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e)
+      if (e * kWideThreads + t < nB) mb = max(mb, bits[e]);
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    if ((t & 31) == 0) cnt[0][t >> 5] = mb;
+    __syncthreads();
+    for (int w = 0; w < kWideThreads / 32; ++w) tb = max(tb, cnt[0][w]);
+    need = 1;
+    __syncthreads();
+  } else if (!none) {
+    uint32_t lo = 0, hi = kInvalidBits;                     // invariant: S(lo) >= T > S(hi)
+    while (hi - lo > 1) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      uint64_t s4[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) s4[e & 3] += (bits[e] >= mid) ? weight(e) : 0;
+      const uint64_t sum = cta_sum_u64((s4[0] + s4[1]) + (s4[2] + s4[3]), red[step++ & 1]);
+      if (sum >= T) lo = mid;
+      else hi = mid;
+    }
+    tb = lo;
+    uint64_t above = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) above += (bits[e] > tb) ? weight(e) : 0;
+    above = cta_sum_u64(above, red[step++ & 1]);
+    const uint64_t ww = kind == 0 ? fixed_weight(tb) : 1ull;
+    need = static_cast<uint32_t>((T - above + ww - 1) / ww);
+  }
+  // emit in ascending index order: chunk e holds indices e*256 .. e*256 + 255
+  uint32_t base = 0, ties_before = 0;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const int idx = e * kWideThreads + t;
+    const bool elig = idx < nB && idx != diag;
+    const bool tie = !none && elig && bits[e] == tb;
+    uint32_t ttot, ktot;
+    const uint32_t rank = ties_before + cta_prefix(tie, cnt[e & 1], ttot);
+    const bool keep = (idx == diag && idx < nB) || (!none && elig && (bits[e] > tb || (tie && rank < need)));
+    const uint32_t pos = base + cta_prefix(keep, cnt[2 + (e & 1)], ktot);
+    if (keep) out[pos] = idx;
+    base += ktot;
+    ties_before += ttot;
+  }
+  if (t == 0) counts[row] = static_cast<int32_t>(base);
+}
+
 // ---------------------------------------------------------------- head scope
 // Weighted MSD radix select over 30 significant bits in three 10-bit digits.
 struct HeadState {
@@ -402,7 +549,7 @@ __global__ void head_emit_kernel(const float* __restrict__ scores, int G, int nB
 // every warp decides 8 token rows in flat order (ties ranked across the head
 // by the scanned per-row tie counts), the keep bits are transposed in shared
 // memory, then the non-empty entries are compacted in ascending order.
-constexpr int kTokMaxB = 1024;                // nB bound of per-token scope
+constexpr int kTokMaxB = 4096;                // nB bound of per-token scope
 __global__ void __launch_bounds__(256) token_emit_kernel(const float* __restrict__ scores, int G, int nQ, int nB,
                                                          const HeadState* __restrict__ st,
                                                          const int32_t* __restrict__ tiebase,
@@ -937,6 +1084,20 @@ __global__ void __launch_bounds__(256) domain_select_kernel(const float* __restr
 }  // namespace
 
 // skip_head: see select_row_kernel (NULL for plain row scope)
+static cudaError_t launch_select_wide(const float* scores, int R, int nB, int kind, uint32_t P, int keep_all, int k,
+                                      const int32_t* head_floor, lbsa_blockset* bs, const int32_t* skip_head,
+                                      cudaStream_t s) {
+  if (nB > 4096) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(R));
+#define LBSA_WIDE(EPT)                                                                                             \
+  select_wide_kernel<EPT><<<grid, kWideThreads, 0, s>>>(scores, R, nB, kind, P, keep_all, k, head_floor, bs->counts, \
+                                                         bs->cols, bs->status, skip_head)
+  if (nB <= 2048) LBSA_WIDE(8);
+  else LBSA_WIDE(16);
+#undef LBSA_WIDE
+  return cudaGetLastError();
+}
+
 static cudaError_t launch_select_row_skip(const float* scores, int R, int nB, double p, lbsa_blockset* bs, cudaStream_t s,
                                    const int32_t* skip_head) {
   const uint32_t P = fixed_p(p);
@@ -955,7 +1116,7 @@ static cudaError_t launch_select_row_skip(const float* scores, int R, int nB, do
   else if (nB <= 256) LBSA_SEL(8);
   else if (nB <= 512) LBSA_SEL(16);
   else if (nB <= 1024) LBSA_SEL(32);
-  else return cudaErrorInvalidValue;
+  else return launch_select_wide(scores, R, nB, 0, P, keep_all, 0, nullptr, bs, skip_head, s);
 #undef LBSA_SEL
   return cudaGetLastError();
 }
@@ -977,7 +1138,7 @@ cudaError_t launch_select_rank(const float* scores, int R, int nB, int mode, int
   else if (nB <= 256) LBSA_RANK(8);
   else if (nB <= 512) LBSA_RANK(16);
   else if (nB <= 1024) LBSA_RANK(32);
-  else return cudaErrorInvalidValue;
+  else return launch_select_wide(scores, R, nB, mode == 0 ? 1 : 2, 0u, 0, k, head_floor, bs, nullptr, s);
 #undef LBSA_RANK
   return cudaGetLastError();
 }

@@ -165,7 +165,7 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
  *       floor is K = ceil(sum_i v_i c_i / sum_i v_i) with v_i the valid tokens
  *       of query block i, min(block, n_valid - i * block); row i keeps the
  *       first max(c_i, min(K, nB)) blocks of its ranked order.  k unused.
- * Ranked order: score descending, then key-block id ascending.  nB <= 1024.
+ * Ranked order: score descending, then key-block id ascending.  nB <= 4096.
  * Invalid scores are handled as by lbsa_select.
  *   n_valid  valid tokens: (nB - 1) * block < n_valid <= nB * block
  *   p        in (0, 1] (LBSA_RULE_TOPP_FLOOR)
@@ -179,7 +179,7 @@ int lbsa_select_rule(const float* scores, int32_t B, int32_t H, int32_t nB, int3
  * here over its (query token, key block) pairs, the pairs of the
  * LBSA_SCORE_MEANPOOL_TOKEN scores; threshold tau; tokens may keep nothing).
  *   scores   fp32 [B, H, n_valid, nB] contiguous device array, 0 <= x < 2
- *   n_valid  valid tokens; nB = ceil(n_valid / 64) <= 1024
+ *   n_valid  valid tokens; nB = ceil(n_valid / 64) <= 4096
  *   block    must be 64 (a query block's tokens fit one 64-bit mask)
  *   p        in (0, 1]
  *   out      receives a new blockset (scope LBSA_SCOPE_TOKEN, free with
@@ -227,7 +227,7 @@ int lbsa_select_tokens(const float* scores, int32_t B, int32_t H, int32_t n_vali
  * score keeps every block of its rows and sets LBSA_ERR_INVALID_SCORES (a
  * head with a NaN or negative score has a NaN entropy and is never routed).
  * Scratch: B*H*ceil(nB/8) fp64 partial entropy sums and the domain tables,
- * from the library pool; nB <= 1024, H <= 4096 and B*H <= 65535; a pool's
+ * from the library pool; nB <= 4096, H <= 4096 and B*H <= 65535; a pool's
  * min(group, H) * nB scores must fit 200 KiB of shared memory, else
  * LBSA_ERR_UNSUPPORTED. */
 int lbsa_select_routed(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,

@@ -79,7 +79,7 @@ def test_select_rejects_bad_scope_block_and_size():
     h = ctypes.c_void_p()
     assert lib.lbsa_select(FAKE, 1, 1, 4, 64, 0.9, 5, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select(FAKE, 1, 1, 4, 32, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
-    assert lib.lbsa_select(FAKE, 1, 1, 2000, 64, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select(FAKE, 1, 1, 4097, 64, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
     assert lib.lbsa_select(FAKE, 1, 1, 0, 64, 0.9, 0, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select(FAKE, 1, 1, 4, 64, 0.9, 0, None, None) == lbsa.LBSA_ERR_INVALID_ARG
 
@@ -128,7 +128,7 @@ def test_select_tokens_rejects_bad_block_p_and_size():
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 128, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.0, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 1.5, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
-    assert lib.lbsa_select_tokens(p, 1, 1, 64 * 1025, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_select_tokens(p, 1, 1, 64 * 4097, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_UNSUPPORTED
     assert lib.lbsa_select_tokens(p, 0, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(p, 1, 1, 256, 64, 0.25, None, None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_select_tokens(None, 1, 1, 256, 64, 0.25, ctypes.byref(h), None) == lbsa.LBSA_ERR_INVALID_ARG
@@ -154,7 +154,7 @@ def test_select_routed_rejects_bad_args():
     assert call(group=0) == lbsa.LBSA_ERR_INVALID_ARG
     assert call(B=0) == lbsa.LBSA_ERR_INVALID_ARG
     assert call(B=20, H=4000) == lbsa.LBSA_ERR_UNSUPPORTED                # B*H > 65535
-    assert call(nB=1025, group=1) == lbsa.LBSA_ERR_UNSUPPORTED             # past the row kernel's width
+    assert call(nB=4097, group=1) == lbsa.LBSA_ERR_UNSUPPORTED             # past the wide row kernel
     assert call(H=4097) == lbsa.LBSA_ERR_UNSUPPORTED
     assert call(H=64, nB=1024, group=64) == lbsa.LBSA_ERR_UNSUPPORTED   # a 64-head pool of 1024 blocks: 256 KiB
     assert call(out=None) == lbsa.LBSA_ERR_INVALID_ARG
