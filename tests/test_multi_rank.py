@@ -8,7 +8,8 @@ import pytest
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from block_sparse_attention_16_b200.multi import lpt_shards, max_over_ranks, shard_loads, barrier
+from block_sparse_attention_16_b200.multi import (barrier, lpt_shards, max_over_ranks, run_sharded_layer,
+                                                 shard_loads)
 
 
 def _free_port():
@@ -70,3 +71,64 @@ def test_single_process_helpers_are_identity():
     assert lpt_shards([5, 5, 5], 1) == [[0, 1, 2]]
     with pytest.raises(ValueError):
         lpt_shards([1], 0)
+
+
+# ---------------------------------------------------------------- one layer split over two ranks
+def _tiny_layer():
+    """A tiny fp64 layer (B=2, H=3, 256 tokens, d=64), its oracle blockset at
+    p = 0.9, and the kept pairs per (batch, head) unit."""
+    import torch
+    import oracle
+    rng = np.random.default_rng(7)
+    q, k, v = (torch.from_numpy(rng.standard_normal((2, 3, 256, 64))) for _ in range(3))
+    masses = oracle.block_mass(q.numpy(), k.numpy(), 256, 64)
+    rp, col = oracle.select_contract(masses.astype(np.float32), 0.9, "row")
+    weights = np.diff(rp).reshape(6, 4).sum(1).tolist()
+    return q, k, v, rp, col, weights
+
+
+def _oracle_units(rp, col):
+    """The host stand-in of the GPU attention: the oracle's block-sparse
+    attention of each listed unit with its rows of the CSR."""
+    import torch
+    import oracle
+
+    def compute(qu, ku, vu, units):
+        outs = []
+        for n, u in enumerate(units):
+            a = rp[u * 4]
+            urp, ucol = rp[u * 4:u * 4 + 5] - a, col[a:rp[u * 4 + 4]]
+            o, _ = oracle.sparse_attention(qu[n:n + 1][None].numpy(), ku[n:n + 1][None].numpy(),
+                                           vu[n:n + 1][None].numpy(), 256, 64, urp, ucol)
+            outs.append(torch.from_numpy(o[0, 0]))
+        return torch.stack(outs) if outs else qu[:0]
+    return compute
+
+
+def _layer_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, rp, col, weights = _tiny_layer()
+        out = run_sharded_layer(q, k, v, weights, _oracle_units(rp, col))
+        units, mine = run_sharded_layer(q, k, v, weights, _oracle_units(rp, col), gather=False)
+        np.save(os.path.join(out_dir, f"full{rank}.npy"), out.numpy())
+        np.save(os.path.join(out_dir, f"units{rank}.npy"), np.array(units))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_layer_on_two_gloo_ranks_equals_one_process(tmp_path):
+    """Shard by LPT on kept pairs, compute each rank's heads, all_gather: every
+    rank ends with exactly the one-process layer output."""
+    q, k, v, rp, col, weights = _tiny_layer()
+    ref = _oracle_units(rp, col)(q.reshape(6, 256, 64), k.reshape(6, 256, 64), v.reshape(6, 256, 64),
+                                 list(range(6))).reshape(2, 3, 256, 64).numpy()
+    mp.start_processes(_layer_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    shards = lpt_shards(weights, 2)
+    for r in range(2):
+        assert np.array_equal(np.load(tmp_path / f"full{r}.npy"), ref)
+        assert np.load(tmp_path / f"units{r}.npy").tolist() == shards[r]
+    assert sorted(shards[0] + shards[1]) == list(range(6)) and shards[0] and shards[1]
