@@ -90,8 +90,10 @@ struct PPLayout {
   // q_full[2], pair_full[NPAIR], pair_empty[NPAIR], s_full[2], p_full[2], o_final[2], drain
   static constexpr int NBAR = 2 + 2 * NPAIR + 7;
   // [0] tmem base [1] abort [2] entries kept by both tiles [3] by A only [4] by B only
+  // [5] the fused dense step's strip slot (-1: none)
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_BITMAP = OFF_MISC + 32;       // 4 bitmaps of nB bits (A0, A1, B0, B1)
+  static constexpr int OFF_LSE = (OFF_MISC + 32 + 15) / 16 * 16;   // fused dense step: [2 tiles][128 rows] row lse (log2)
+  static constexpr int OFF_BITMAP = OFF_LSE + 2 * kBM * 4;  // 4 bitmaps of nB bits (A0, A1, B0, B1)
   __host__ __device__ static int words(int nB) { return (nB + 31) >> 5; }
   __host__ __device__ static int sched_off(int nB) { return OFF_BITMAP + 4 * words(nB) * 4; }
   // merged list: nB uint16 entries (bits 0-11 key block; bit 12 + 2*tile + half: that
@@ -252,6 +254,31 @@ __device__ __forceinline__ void max_half0(const uint32_t (&r)[128], float (&mx8)
     mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(r[c]), __uint_as_float(r[c + 1]));
 }
 
+// Warp transpose-reduce: lane l holds x[0..31] (one partial per key block);
+// afterwards x[0] of lane l is the sum over the 32 lanes of x[l].  Five levels;
+// at the level of width w a lane keeps the half of its values that its lane bit w
+// selects, sends the other half to lane ^ w and adds what it receives.
+__device__ __forceinline__ void warp_transpose_reduce32(float (&x)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? x[i] : x[i + w];
+      const float keep = upper ? x[i + w] : x[i];
+      x[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+}
+
+// The row sum of the packed partial sums (a fixed order).
+__device__ __forceinline__ float hsum4(const unsigned long long (&sum4)[4]) {
+  float s8[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) u64_as_f2(sum4[i], s8[2 * i], s8[2 * i + 1]);
+  return ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+}
+
 __device__ __forceinline__ float max8(const float (&mx8)[8]) {
   return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])), fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
 }
@@ -264,7 +291,7 @@ __device__ __forceinline__ float raise_max(float m, float mx) {
   return mx > m + 8.0f ? ceilf(mx) : m;
 }
 
-template <int D>
+template <int D, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const AttendArgs args, float scale_log2) {
@@ -327,7 +354,35 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
                     (tileA + t) * kBM, h, bb);
     }
   }
-  {
+  if (FUSED) {
+    // dense step: every key block for every query block of the CTA
+    for (int i = tid; i < nwords; i += kThreads) {
+      const uint32_t all = (i == nwords - 1 && (nB & 31)) ? ((1u << (nB & 31)) - 1u) : 0xffffffffu;
+      bm[i] = all;
+      bm[nwords + i] = all;
+      bm[2 * nwords + i] = hasB ? all : 0u;
+      bm[3 * nwords + i] = hasB ? all : 0u;
+    }
+    if (tid == 0) {
+      // a strip slot: at most one CTA per SM holds TMEM at a time and each holds one
+      // slot, so a free one exists; the probe is bounded all the same
+      int slot = -1;
+      const uint64_t t0 = globaltimer_ns();
+      for (int i = (blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) % args.n_slots;;
+           i = (i + 1) % args.n_slots) {
+        if (atomicCAS(args.slots + i, 0, 1) == 0) {
+          slot = i;
+          break;
+        }
+        if (globaltimer_ns() - t0 > static_cast<uint64_t>(args.wait_limit)) {
+          raise_status(args.status, LBSA_ERR_TIMEOUT);
+          break;
+        }
+      }
+      __threadfence();
+      misc[5] = static_cast<uint32_t>(slot);
+    }
+  } else {
     // query blocks: b = 64: A0 = 4u, A1 = 4u+1, B0 = 4u+2, B1 = 4u+3; b = 128: A = 2u, B = 2u+1
     const long long hrow = (static_cast<long long>(bb) * args.H + h) * nB;
     const int per_tile = (blk == 64) ? 2 : 1;
@@ -397,9 +452,11 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       }
     }
     if (lane == 0) {
-      misc[2] = static_cast<uint32_t>(tot[0]);
-      misc[3] = static_cast<uint32_t>(tot[1]);
-      misc[4] = static_cast<uint32_t>(tot[2]);
+      // fused step without a strip slot: no steps (the call has failed)
+      const bool none = FUSED && static_cast<int>(misc[5]) < 0;
+      misc[2] = none ? 0u : static_cast<uint32_t>(tot[0]);
+      misc[3] = none ? 0u : static_cast<uint32_t>(tot[1]);
+      misc[4] = none ? 0u : static_cast<uint32_t>(tot[2]);
     }
   }
   tc_fence_before();
@@ -560,6 +617,12 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
     const uint32_t o_col = 256 + t * 128;
     const int n_steps = t ? nSB : nSA;
     const int kbit = 12 + 2 * t + rh;          // this row's keep bit in a list entry
+    // fused dense step: this CTA's strip, [tile][64-key chunk][row] log-sum-exp (log2 units)
+    const int n_chunks = (args.N_valid + 63) / 64;
+    const int slot = FUSED ? static_cast<int>(misc[5]) : -1;
+    // this row's column of its tile's strip: an element offset into the scratch
+    // (below 2^31: at most 2 x SM count x 128 x 8192 floats), -1 without a slot
+    const int soff = (FUSED && slot >= 0) ? ((slot * 2 + t) * n_chunks * kBM + row) : -1;
     float m = -INFINITY;                       // running max (log2 units, an integer), possibly stale by < 8
     float l = 0.f;
     bool alive = true;
@@ -631,6 +694,13 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         for (int i = 0; i < 4; ++i) sum4[i] = ffma2(sum4[i], f2, 0ull);
       }
       tmem_st32(t_lane + s_col, pk);
+      float sum_h0 = 0.f;
+      if (FUSED) {
+        // the fused step keeps the two 64-key halves' sums apart
+        sum_h0 = hsum4(sum4);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum4[i] = 0ull;
+      }
       {
         const float mu = (m == -INFINITY) ? 0.f : m;
         const unsigned long long nm2 = f2_as_u64(-mu, -mu);
@@ -638,6 +708,16 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         else exp_half<0, 1, false>(r, sc2, nm2, sum4, pk, mx8);
       }
       tmem_st32(t_lane + s_col + 32, pk);
+      float sum_step = hsum4(sum4);
+      // fused step: each 64-key chunk's log-sum-exp (log2 units), chunks 2u and 2u + 1
+      // of merged-list step u (the dense list walks every key block in order); stored
+      // once P is published, so the stores never hold up the arrival
+      float lse_c0 = 0.f, lse_c1 = 0.f;
+      if (FUSED) {
+        lse_c0 = m + __log2f(sum_h0);
+        lse_c1 = m + __log2f(sum_step);
+        sum_step += sum_h0;
+      }
       // O and the row sum of earlier steps, rescaled to the new max (exactly)
       const bool need = m_start != -INFINITY && m != m_start;
       if (__any_sync(0xffffffffu, need)) {
@@ -655,14 +735,16 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
         }
         l *= f;
       }
-      float sum8[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) u64_as_f2(sum4[i], sum8[2 * i], sum8[2 * i + 1]);
-      l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      l += sum_step;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full + t);
+      if (FUSED && soff >= 0) {
+        const int c0 = 2 * ts.step(t, s);
+        if (c0 < n_chunks) args.fscratch[soff + c0 * kBM] = lse_c0;
+        if (c0 + 1 < n_chunks) args.fscratch[soff + (c0 + 1) * kBM] = lse_c1;
+      }
     }
     // ---- epilogue: O / l -> out, lse
     bool ok_o = alive && n_steps > 0 && !*abort_flag;
@@ -699,10 +781,67 @@ attend_pp_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_consta
       const float v = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       args.lse[(static_cast<long long>(bb) * args.H + h) * args.N_valid + grow] = v;
     }
+    if (FUSED) {
+      // exact block masses (LoSA abstract): 2^(L[r,c] - lse_r) is row r's share on
+      // chunk c.  Each warp of the tile takes groups of 32 key blocks; lane l reads
+      // rows l, l+32, l+64, l+96 of each chunk (coalesced), sums per query block, and
+      // a transpose-reduce leaves key block 32g + l's sums in lane l.  Invalid rows
+      // have lse = +inf and add nothing.
+      float* lse_s = reinterpret_cast<float*>(smem + L::OFF_LSE) + t * kBM;
+      lse_s[row] = (valid && l > 0.f) ? m + __log2f(l) : INFINITY;
+      named_bar_sync(1 + t, kBM);
+      if (soff >= 0 && (t == 0 || hasB) && __all_sync(0xffffffffu, ok_o)) {
+        const float* st = args.fscratch + (soff - row) + lane;     // the tile's strip, this lane's row
+        const long long hrow = (static_cast<long long>(bb) * args.H + h) * nB;
+        float ls[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ls[j] = lse_s[lane + 32 * j];
+        for (int g = warp & 3; g * 32 < nB; g += 4) {
+          float x0[32], x1[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int kb = g * 32 + j;
+            float a0 = 0.f, a1 = 0.f;
+            if (blk == 64) {
+              if (kb < nB) {
+                const float* sc = st + static_cast<long long>(kb) * kBM;
+                a0 = ex2(sc[0] - ls[0]) + ex2(sc[32] - ls[1]);
+                a1 = ex2(sc[64] - ls[2]) + ex2(sc[96] - ls[3]);
+              }
+            } else {
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                if (2 * kb + cc < n_chunks) {
+                  const float* sc = st + static_cast<long long>(2 * kb + cc) * kBM;
+                  a0 += (ex2(sc[0] - ls[0]) + ex2(sc[32] - ls[1])) + (ex2(sc[64] - ls[2]) + ex2(sc[96] - ls[3]));
+                }
+              }
+            }
+            x0[j] = a0;
+            x1[j] = a1;
+          }
+          warp_transpose_reduce32(x0, lane);
+          if (blk == 64) warp_transpose_reduce32(x1, lane);
+          const int kb = g * 32 + lane;
+          if (kb < nB) {
+            for (int q = 0; q < (blk == 64 ? 2 : 1); ++q) {
+              const int qb = (blk == 64) ? 2 * (tileA + t) + q : tileA + t;
+              if (qb >= nB) continue;
+              const int rv = min(blk, args.N_valid - qb * blk);
+              args.scores[(hrow + qb) * nB + kb] = (q ? x1[0] : x0[0]) / static_cast<float>(rv);
+            }
+          }
+        }
+      }
+    }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (FUSED && tid == 0 && static_cast<int>(misc[5]) >= 0) {
+    __threadfence();                          // the strip's last readers are done
+    atomicExch(args.slots + misc[5], 0);
+  }
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(misc[0], kTmemCols);
@@ -716,9 +855,10 @@ bool attend_pp_supported(const AttendArgs& a) {
   return a.masks == nullptr && a.nB <= kMaxBlocks && (a.d == 64 || a.d == 128) && (a.block == 64 || a.block == 128);
 }
 
-cudaError_t launch_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                                  const AttendArgs& a, cudaStream_t s) {
-  if (!attend_pp_supported(a)) return cudaErrorInvalidValue;
+namespace {
+template <bool FUSED>
+cudaError_t launch_pp(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv, const AttendArgs& a,
+                      cudaStream_t s) {
   const int tiles = (a.N_valid + kBM - 1) / kBM;
   dim3 grid((tiles + 1) / 2, a.H, a.B);
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
@@ -733,8 +873,44 @@ cudaError_t launch_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, 
     kern<<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
     return cudaGetLastError();
   };
-  if (a.d == 128) return go(attend_pp_kernel<128>, PPLayout<128>::bytes(a.nB), regs_launch_min<128>());
-  return go(attend_pp_kernel<64>, PPLayout<64>::bytes(a.nB), regs_launch_min<64>());
+  if (a.d == 128) return go(attend_pp_kernel<128, FUSED>, PPLayout<128>::bytes(a.nB), regs_launch_min<128>());
+  return go(attend_pp_kernel<64, FUSED>, PPLayout<64>::bytes(a.nB), regs_launch_min<64>());
+}
+
+int sm_count() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+}  // namespace
+
+cudaError_t launch_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                  const AttendArgs& a, cudaStream_t s) {
+  if (!attend_pp_supported(a)) return cudaErrorInvalidValue;
+  return launch_pp<false>(tq, tk, tv, a, s);
+}
+
+size_t score_attend_pp_workspace_bytes(int N_valid, int* n_slots, size_t* flag_bytes) {
+  // one CTA per SM holds TMEM at a time, and a CTA takes its slot while it holds TMEM
+  const int slots = sm_count();
+  if (n_slots) *n_slots = slots;
+  const size_t flags = (static_cast<size_t>(slots) * sizeof(int32_t) + 255) / 256 * 256;   // slot flags first
+  if (flag_bytes) *flag_bytes = flags;
+  const size_t n_chunks = (N_valid + 63) / 64;
+  return flags + static_cast<size_t>(slots) * 2 * kBM * n_chunks * sizeof(float);
+}
+
+cudaError_t launch_score_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                        const AttendArgs& a, cudaStream_t s) {
+  if (a.masks != nullptr || a.nB > kMaxBlocks || a.n_slots < 1 || !a.slots || !a.fscratch || !a.scores ||
+      !(a.d == 64 || a.d == 128) || !(a.block == 64 || a.block == 128))
+    return cudaErrorInvalidValue;
+  return launch_pp<true>(tq, tk, tv, a, s);
 }
 
 }  // namespace lbsa

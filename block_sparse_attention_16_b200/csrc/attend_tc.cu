@@ -96,7 +96,7 @@ __device__ __forceinline__ Bars make_bars(uint8_t* base) {
   return r;
 }
 
-template <int D, bool FUSED, bool MASKED>
+template <int D, bool MASKED>
 __global__ void __launch_bounds__(kThreads, 2)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                    const __grid_constant__ CUtensorMap tmap_v, const AttendArgs args, float scale_log2) {
@@ -168,31 +168,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
 
   const int qb0 = (blk == 64) ? 2 * tile : tile;
   const int qb1 = (blk == 64 && 2 * tile + 1 < nB) ? 2 * tile + 1 : -1;
-  if (FUSED) {
-    // dense step: every key block, both row halves
-    for (int i = tid; i < nB; i += kThreads) sched[i] = static_cast<uint32_t>(i) | (3u << 30);
-    if (tid == 0) {
-      misc[2] = static_cast<uint32_t>(nB);
-      // a strip slot: at most two CTAs per SM hold TMEM at a time and each holds
-      // one slot, so a free one exists; the probe is bounded all the same
-      int slot = -1;
-      const uint64_t t0 = globaltimer_ns();
-      for (int i = (blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) % args.n_slots;;
-           i = (i + 1) % args.n_slots) {
-        if (atomicCAS(args.slots + i, 0, 1) == 0) {
-          slot = i;
-          break;
-        }
-        if (globaltimer_ns() - t0 > static_cast<uint64_t>(args.wait_limit)) {
-          raise_status(args.status, LBSA_ERR_TIMEOUT);
-          break;
-        }
-      }
-      __threadfence();
-      misc[3] = static_cast<uint32_t>(slot);
-      if (slot < 0) misc[2] = 0;              // no steps: the CTA leaves without work
-    }
-  } else {
+  {
     // both rows' counts, then both lists, with their loads in flight together
     const long long row0 = (static_cast<long long>(bb) * args.H + h) * nB + qb0;
     const long long row1 = row0 + 1;
@@ -223,7 +199,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
     }
   }
   __syncthreads();
-  if (!FUSED && warp == 0) {
+  if (warp == 0) {
     // each lane owns a contiguous run of bitmap words; exclusive scan of popcounts
     const int per = (nwords + 31) / 32;
     const int w0 = lane * per;
@@ -254,11 +230,6 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
   const uint32_t tmem = misc[0];
   const int n_steps = static_cast<int>(misc[2]) * spb;
   const long long wl = args.wait_limit;
-  // fused dense step: this CTA's strip (log-sum-exp per row and 64-key chunk) and partials
-  const int n_chunks = (args.N_valid + BK - 1) / BK;
-  const int slot = FUSED ? static_cast<int>(misc[3]) : -1;
-  float* strip = (FUSED && slot >= 0) ? args.fscratch + static_cast<long long>(slot) * (BM + 4) * n_chunks : nullptr;
-  float* part = strip ? strip + static_cast<long long>(BM) * n_chunks : nullptr;     // [4][n_chunks]
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -459,7 +430,6 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
       l += bsum;
-      if (FUSED && strip && s < n_chunks) strip[static_cast<long long>(s) * BM + row] = m + __log2f(bsum);   // chunk s's log-sum-exp
       if (s >= 2 && !mbar_wait(bars.o_done + sb, ((s - 2) >> 1) & 1, wl, args.status, abort_flag)) {
         alive = false;
         break;
@@ -505,56 +475,10 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_cons
       const float v = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       args.lse[(static_cast<long long>(bb) * args.H + h) * args.N_valid + grow] = v;
     }
-    if (FUSED && strip) {
-      // exact block masses (LoSA abstract): 2^(L[r,c] - lse_r) is row r's mass on
-      // chunk c; summed over the warp's rows, then over the block's rows / |rows|
-      const float lse2 = m + __log2f(l);
-      for (int ch0 = 0; ch0 < n_chunks; ch0 += 16) {
-        float Lv[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          Lv[u] = (ch0 + u < n_chunks) ? strip[static_cast<long long>(ch0 + u) * BM + row] : -INFINITY;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          if (ch0 + u >= n_chunks) break;
-          float w = valid ? ex2(Lv[u] - lse2) : 0.f;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
-          if (lane == 0) part[warp * n_chunks + ch0 + u] = w;
-        }
-      }
-      named_bar_sync(1, 128);
-      const long long hrow = (static_cast<long long>(bb) * args.H + h) * nB;
-      if (blk == 64) {
-        for (int o = tid; o < 2 * nB; o += 128) {
-          const int hf = o / nB, kb = o % nB;
-          const int qb = 2 * tile + hf;
-          if (qb >= nB) continue;
-          const int rv = min(64, args.N_valid - qb * 64);
-          args.scores[(hrow + qb) * nB + kb] =
-              (part[(2 * hf) * n_chunks + kb] + part[(2 * hf + 1) * n_chunks + kb]) / static_cast<float>(rv);
-        }
-      } else {
-        const int qb = tile;
-        const int rv = min(128, args.N_valid - qb * 128);
-        for (int kb = tid; kb < nB; kb += 128) {
-          float w = 0.f;
-          for (int hf = 0; hf < 2; ++hf) {
-            const int c = 2 * kb + hf;
-            if (c < n_chunks) w += (part[c] + part[n_chunks + c]) + (part[2 * n_chunks + c] + part[3 * n_chunks + c]);
-          }
-          args.scores[(hrow + qb) * nB + kb] = w / static_cast<float>(rv);
-        }
-      }
-    }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (FUSED && tid == 0 && slot >= 0) {
-    __threadfence();                          // the strip's last readers are done
-    atomicExch(args.slots + slot, 0);
-  }
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -578,54 +502,10 @@ cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, con
     return cudaGetLastError();
   };
   if (a.d == 128)
-    return masked ? go(attend_bf16_kernel<128, false, true>, Layout<128>::bytes(a.nB, true))
-                  : go(attend_bf16_kernel<128, false, false>, Layout<128>::bytes(a.nB));
-  return masked ? go(attend_bf16_kernel<64, false, true>, Layout<64>::bytes(a.nB, true))
-                : go(attend_bf16_kernel<64, false, false>, Layout<64>::bytes(a.nB));
-}
-
-int g_fused_sms = 0;
-int fused_slots() {
-  if (!g_fused_sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_fused_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_fused_sms <= 0) g_fused_sms = 148;
-  }
-  return 2 * g_fused_sms;                     // CTAs that can hold TMEM at once
-}
-
-size_t score_attend_bf16_workspace_bytes(int N_valid, int* n_slots, size_t* flag_bytes) {
-  const int slots = fused_slots();
-  if (n_slots) *n_slots = slots;
-  const size_t flags = (static_cast<size_t>(slots) * sizeof(int32_t) + 255) / 256 * 256;   // slot flags first
-  if (flag_bytes) *flag_bytes = flags;
-  const size_t n_chunks = (N_valid + BK - 1) / BK;
-  return flags + static_cast<size_t>(slots) * (BM + 4) * n_chunks * sizeof(float);
-}
-
-cudaError_t launch_score_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                                     const AttendArgs& a, cudaStream_t s) {
-  const int tiles = (a.N_valid + BM - 1) / BM;
-  dim3 grid(tiles, a.H, a.B);
-  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(a.d)));
-  if (a.nB > kMaxBlocks || a.n_slots < 1) return cudaErrorInvalidValue;
-  // at least 80 KB of shared memory: two CTAs per SM at most, as the slot count assumes
-  auto smem_of = [](size_t b) { return b < 80 * 1024 ? static_cast<size_t>(80 * 1024) : b; };
-  if (a.d == 128) {
-    const size_t smem = smem_of(Layout<128>::bytes(a.nB));
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<128, true, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attend_bf16_kernel<128, true, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
-  } else {
-    const size_t smem = smem_of(Layout<64>::bytes(a.nB));
-    cudaError_t e = cudaFuncSetAttribute(attend_bf16_kernel<64, true, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attend_bf16_kernel<64, true, false><<<grid, kThreads, smem, s>>>(*tq, *tk, *tv, a, scale_log2);
-  }
-  return cudaGetLastError();
+    return masked ? go(attend_bf16_kernel<128, true>, Layout<128>::bytes(a.nB, true))
+                  : go(attend_bf16_kernel<128, false>, Layout<128>::bytes(a.nB));
+  return masked ? go(attend_bf16_kernel<64, true>, Layout<64>::bytes(a.nB, true))
+                : go(attend_bf16_kernel<64, false>, Layout<64>::bytes(a.nB));
 }
 
 }  // namespace lbsa

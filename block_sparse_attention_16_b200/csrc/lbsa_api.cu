@@ -284,7 +284,7 @@ int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qk
   if ((rc = device_state(&ds)) != LBSA_OK) return rc;
   int n_slots = 0;
   size_t flag_bytes = 0;
-  const size_t bytes = lbsa::score_attend_bf16_workspace_bytes(desc->N_valid, &n_slots, &flag_bytes);
+  const size_t bytes = lbsa::score_attend_pp_workspace_bytes(desc->N_valid, &n_slots, &flag_bytes);
   Scratch ws;
   if ((rc = scratch_alloc(ds, bytes, s, &ws)) != LBSA_OK) return rc;
   lbsa::AttendArgs a{desc->B, desc->H, desc->N_valid, desc->d, block, nB, nullptr, nullptr, ds->status,
@@ -296,7 +296,7 @@ int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qk
   if ((rc = make_tmap(&tk, k, desc, 64)) != LBSA_OK) return rc;
   if ((rc = make_tmap(&tv, v, desc, 64)) != LBSA_OK) return rc;
   cudaError_t e = cudaMemsetAsync(ws.ptr, 0, flag_bytes, s);     // every strip slot free
-  if (e == cudaSuccess) e = lbsa::launch_score_attend_bf16(&tq, &tk, &tv, a, s);
+  if (e == cudaSuccess) e = lbsa::launch_score_attend_pp_bf16(&tq, &tk, &tv, a, s);
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_score_attend launch");
   return LBSA_OK;
 }

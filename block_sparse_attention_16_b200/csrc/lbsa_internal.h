@@ -34,9 +34,9 @@ struct AttendArgs {
   int64_t ostride_b, ostride_h, ostride_n;   // elements
   float* lse;
   long long wait_limit;
-  // fused dense step only (launch_score_attend_bf16): exact block masses out
+  // fused dense step only (launch_score_attend_pp_bf16): exact block masses out
   float* scores;          // [B, H, nB, nB]
-  float* fscratch;        // n_slots * (128 + 4) * n_chunks floats: per-CTA strips and partials
+  float* fscratch;        // n_slots * 2 * 128 * n_chunks floats: per-CTA strips
   int32_t* slots;         // n_slots flags, zero at launch
   int n_slots;
   // per-token scope (64-token blocks): masks[row * nB + t] is the 64-bit set of
@@ -62,11 +62,12 @@ cudaError_t launch_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, con
 bool attend_pp_supported(const AttendArgs& a);
 cudaError_t launch_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                                   const AttendArgs& a, cudaStream_t s);
-// dense attention that also writes the exact block masses (a.scores); a.counts/cols unused
-cudaError_t launch_score_attend_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                                     const AttendArgs& a, cudaStream_t s);
-// workspace: n_slots int32 flags (flag_bytes, 256-aligned), then the per-slot strips
-size_t score_attend_bf16_workspace_bytes(int N_valid, int* n_slots, size_t* flag_bytes);
+// the fused dense step on the two-tile kernel: dense attention and the exact block
+// masses (a.scores); workspace: n_slots int32 flags (flag_bytes, 256-aligned), then
+// per slot 2 x 128 x ceil(N_valid / 64) floats of strips
+size_t score_attend_pp_workspace_bytes(int N_valid, int* n_slots, size_t* flag_bytes);
+cudaError_t launch_score_attend_pp_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                                        const AttendArgs& a, cudaStream_t s);
 cudaError_t launch_score_exact_bf16(const CUtensorMap* tq, const CUtensorMap* tk, const ScoreArgs& a,
                                     cudaStream_t s);
 size_t score_exact_bf16_workspace_bytes(int B, int H, int N_valid);

@@ -37,6 +37,26 @@ def test_fused_dense_step_matches_oracle(case):
     assert_csr_equal(gpu_csr(bs), oracle.select_contract(host(scores), 0.9, "row"))
 
 
+def test_fused_dense_step_many_key_blocks():
+    """128-token blocks, nB = 153 > 128 (each mass thread takes two key blocks),
+    ragged last block: every mass against the exact scorer, sampled query blocks
+    against the fp64 oracle, O against attention over the dense blockset."""
+    wl = small_workload("f128_nb153", 1, 2, 128, (5, 30, 130), 128, dtype="bf16", wid=161)   # 19500 tokens
+    assert wl.n_blocks == 153
+    q, k, v = (x.cuda() for x in make_qkv(wl))
+    scores, out = lbsa.lbsa_score_attend(q, k, v, wl.block)
+    ref_scores = lbsa.lbsa_score(q, k, wl.block)
+    ref_out = lbsa.lbsa_attend(q, k, v, lbsa.lbsa_select(ref_scores, wl.block, 1.0, "row"))
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_device_status() == 0
+    assert_scores_close(host(scores), host(ref_scores))
+    assert_out_close(host(out), host(ref_out), torch.bfloat16)
+    sc = host(scores)
+    for h, qb in ((0, 0), (1, 77), (1, 152)):
+        ref = oracle.block_mass(host(q[:, h:h + 1]), host(k[:, h:h + 1]), wl.n_valid, wl.block, qblocks=[qb])
+        assert_scores_close(sc[:, h:h + 1, qb:qb + 1], ref)
+
+
 def test_fused_dense_step_on_the_wan_layer():
     """Full Wan-like layer: masses agree with the scorer's; O agrees with attention over
     the dense blockset (a different kernel, so within the bf16 tolerance, not bit for bit)
