@@ -572,7 +572,9 @@ def load_traffic(kernel):
 
 def run_profile(kernel):
     """A small case for ncu: 6 heads of the Wan-like layer (151 MB of Q/K/V, more
-    than L2), one warm-up pass of the path, then two launches of `kernel`; or,
+    than L2), one warm-up pass of the path, then two launches of `kernel`
+    ("dense": attention over the p = 1 blockset, the two-tile kernel; "fused":
+    the fused dense step); or,
     for "proxy", one mean-pooled proxy call per partition on the full shape; for
     "token", one call of each per-token proxy stage on the full shape (3D tiles)."""
     import dataclasses
@@ -637,9 +639,14 @@ def run_profile(kernel):
     scores = lbsa.lbsa_score(qp, kp, wl.block)
     bs = lbsa.lbsa_select(scores, wl.block, P, "row")
     lbsa.lbsa_attend(qp, kp, vp, bs)
+    dense = lbsa.lbsa_select(scores, wl.block, 1.0, "row") if kernel == "dense" else None
     for _ in range(2):
         if kernel == "attend":
             lbsa.lbsa_attend(qp, kp, vp, bs)
+        elif kernel == "dense":
+            lbsa.lbsa_attend(qp, kp, vp, dense)
+        elif kernel == "fused":
+            lbsa.lbsa_score_attend(qp, kp, vp, wl.block)
         elif kernel == "score":
             lbsa.lbsa_score(qp, kp, wl.block, scores=scores)
         elif kernel == "select":
@@ -874,7 +881,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="leave out the measurements beside the contract's timed calls (dense, step 0, configs 0-4)")
     ap.add_argument("--clocks-csv", default=None, help="where the nvidia-smi clock samples go (default under /tmp)")
-    ap.add_argument("--profile", choices=["attend", "score", "select", "proxy", "token", "routed"],
+    ap.add_argument("--profile", choices=["attend", "dense", "fused", "score", "select", "proxy", "token", "routed"],
                     help="run the small ncu case for one kernel instead of the benchmark")
     ap.add_argument("--sweep", action="store_true", help="per-stage timings on every workload (not the contract line)")
     args = ap.parse_args()

@@ -57,10 +57,19 @@ __device__ __forceinline__ uint64_t threshold_T(uint64_t W, uint32_t Pfix) {
 // One warp per row of nB scores; lane l holds elements l, l+32, ...
 // skip_head (NULL for plain row scope): rows of heads with skip_head[h] >= 0
 // (pooled heads of the routed scope) are left to the domain kernel.
+// The bisection runs in two phases.  While more than 32 weighted elements lie
+// in the bracket [lo, hi), every step sums all of the row's weights at or
+// above mid; each weight carries the element count in its low 11 bits, so the
+// same exact sum also gives the bracket's population.  Then the bracket's
+// elements are compacted to one a lane and the remaining steps sum only
+// those, on top of S at the bracket's upper end.  The result is the bisection's.
+constexpr int kRowThreads = 64;
 template <int EPL>
-__global__ void select_row_kernel(const float* __restrict__ scores, int R, int nB, uint32_t Pfix, int keep_all,
-                                  int32_t* __restrict__ counts, int32_t* __restrict__ cols,
-                                  int32_t* __restrict__ status, const int32_t* __restrict__ skip_head) {
+__global__ void __launch_bounds__(kRowThreads) select_row_kernel(
+    const float* __restrict__ scores, int R, int nB, uint32_t Pfix, int keep_all, int32_t* __restrict__ counts,
+    int32_t* __restrict__ cols, int32_t* __restrict__ status, const int32_t* __restrict__ skip_head) {
+  __shared__ uint32_t cbits[kRowThreads / 32][32];
+  __shared__ unsigned long long cw[kRowThreads / 32][32];
   const int lane = threadIdx.x & 31;
   const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (row >= R) return;
@@ -68,7 +77,7 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + row * nB;
   int32_t* out = cols + row * nB;
   uint32_t bits[EPL];
-  uint64_t w[EPL];
+  uint64_t wc[EPL];            // (w << 11) | 1 for an element of weight w > 0, else 0 (w < 2^33)
   bool bad = false;
   uint64_t wsum = 0;
 #pragma unroll
@@ -77,8 +86,9 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
     const uint32_t b = (idx < nB) ? __ldg(x + idx) : 0u;
     bad |= (idx < nB) && (b >= kInvalidBits);
     bits[e] = b;
-    w[e] = (idx < nB && b < kInvalidBits) ? fixed_weight(b) : 0;
-    wsum += w[e];
+    const uint64_t w = (idx < nB && b < kInvalidBits) ? fixed_weight(b) : 0;
+    wc[e] = w ? ((w << 11) | 1ull) : 0ull;
+    wsum += wc[e];
   }
   const bool any_bad = __any_sync(0xffffffffu, bad);
   if (any_bad || keep_all) {
@@ -87,7 +97,9 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
     if (lane == 0) counts[row] = nB;
     return;
   }
-  const uint64_t W = warp_sum_u64(wsum);
+  // at most 1024 elements of weight < 2^33: every sum below stays under 2^54
+  const uint64_t Wc = warp_sum_u64(wsum);
+  const uint64_t W = Wc >> 11;
   const uint64_t T = threshold_T(W, Pfix);
   uint32_t tb;
   uint32_t need;
@@ -103,21 +115,58 @@ __global__ void select_row_kernel(const float* __restrict__ scores, int R, int n
     need = 1;
   } else {
     uint32_t lo = 0, hi = kInvalidBits;       // invariant: S(lo) >= T > S(hi)
-    while (hi - lo > 1) {
+    uint64_t S_hi = 0;                        // S(hi)
+    uint32_t c_lo = static_cast<uint32_t>(Wc & 2047u), c_hi = 0;   // weighted elements at or above lo / hi
+    const uint64_t Tc = T << 11;              // S(mid) >= T  <=>  (S(mid) << 11) + count >= Tc
+    while (hi - lo > 1 && c_lo - c_hi > 32) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
       // four independent partial sums: the 64-bit adds do not form one long chain
       uint64_t s4[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) s4[e & 3] += (bits[e] >= mid) ? w[e] : 0;
+      for (int e = 0; e < EPL; ++e) s4[e & 3] += (bits[e] >= mid) ? wc[e] : 0;
       const uint64_t s = warp_sum_u64((s4[0] + s4[1]) + (s4[2] + s4[3]));
-      if (s >= T) lo = mid;
-      else hi = mid;
+      if (s >= Tc) {
+        lo = mid;
+        c_lo = static_cast<uint32_t>(s & 2047u);
+      } else {
+        hi = mid;
+        c_hi = static_cast<uint32_t>(s & 2047u);
+        S_hi = s >> 11;
+      }
+    }
+    if (hi - lo > 1) {
+      // at most 32 weighted elements left in [lo, hi): one a lane
+      const int wi = threadIdx.x >> 5;
+      const uint32_t lt = (1u << lane) - 1u;
+      uint32_t n = 0;
+      const uint32_t span = hi - lo;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const bool act = wc[e] != 0 && bits[e] - lo < span;
+        const uint32_t m = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const uint32_t pos = n + __popc(m & lt);
+          cbits[wi][pos] = bits[e];
+          cw[wi][pos] = wc[e];
+        }
+        n += __popc(m);
+      }
+      __syncwarp();
+      const uint32_t b1 = (lane < static_cast<int>(n)) ? cbits[wi][lane] : 0u;
+      const uint64_t w1 = (lane < static_cast<int>(n)) ? (cw[wi][lane] >> 11) : 0ull;
+      const uint64_t base = S_hi;             // S at the bracket's upper end when compacted
+      while (hi - lo > 1) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        const uint64_t s = base + warp_sum_u64((b1 >= mid) ? w1 : 0ull);
+        if (s >= T) lo = mid;
+        else {
+          hi = mid;
+          S_hi = s;
+        }
+      }
     }
     tb = lo;
-    uint64_t above = 0;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) above += (bits[e] > tb) ? w[e] : 0;
-    above = warp_sum_u64(above);
+    const uint64_t above = S_hi;              // S(tb + 1)
     const uint64_t ww = fixed_weight(tb);     // > 0 because S(tb) > S(tb + 1)
     const uint64_t rest = T - above;
     need = static_cast<uint32_t>((rest + ww - 1) / ww);
@@ -1104,7 +1153,7 @@ static cudaError_t launch_select_row_skip(const float* scores, int R, int nB, do
   const int keep_all = p >= 1.0 ? 1 : 0;
   // two warps (rows) per block: residency is then bounded by registers, not by
   // the block granularity of the register-heavy wide-row instantiations
-  const int threads = 64;
+  const int threads = kRowThreads;
   const long long blocks = (static_cast<long long>(R) * 32 + threads - 1) / threads;
   dim3 grid(static_cast<unsigned>(blocks));
 #define LBSA_SEL(EPL)                                                                                       \
