@@ -108,6 +108,25 @@ int make_tmap(CUtensorMap* map, const void* ptr, const lbsa_qkv_desc* d, int box
   return LBSA_OK;
 }
 
+// A dense bf16 [n3][n2][n1][n0] array (n0 innermost, contiguous) as a 4D tensor
+// map with box 64 x box_rows x 1 x 1 and 128-byte swizzle.
+int make_tmap_4d(CUtensorMap* map, const void* ptr, long long n0, long long n1, long long n2, long long n3,
+                 int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(n0), static_cast<cuuint64_t>(n1), static_cast<cuuint64_t>(n2),
+                        static_cast<cuuint64_t>(n3)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(n0) * 2, static_cast<cuuint64_t>(n0 * n1) * 2,
+                           static_cast<cuuint64_t>(n0 * n1 * n2) * 2};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LBSA_OK;
+}
+
 // Per-device state: a status word for calls without a blockset, and a memory
 // pool that serves blocksets and per-call scratch stream-ordered
 // (cudaMallocFromPoolAsync / cudaFreeAsync).  The pool keeps freed memory
@@ -257,7 +276,18 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
     const int nQ = tokens ? desc->N_valid : nB;
     if ((rc = scratch_alloc(ds, lbsa::meanpool_workspace_bytes(desc->B, desc->H, nB, desc->d, nQ), s, &ws)) != LBSA_OK)
       return rc;
-    e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s);
+    if (tokens && desc->dtype == LBSA_BF16) {
+      // the logits on the tensor cores: Q as the attention reads it, and the bf16
+      // hi / lo terms of the key-block means as a (d, nB, G, 2) map
+      CUtensorMap tq, tkb;
+      if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
+      const long long G = static_cast<long long>(desc->B) * desc->H;
+      if ((rc = make_tmap_4d(&tkb, lbsa::meanpool_split_ptr(ws.ptr), desc->d, nB, G, 2, 128)) != LBSA_OK) return rc;
+      e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s, &tq, &tkb, ds->status,
+                                wait_limit());
+    } else {
+      e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s);
+    }
   }
   if (e != cudaSuccess) return cuda_fail(e, "lbsa_score launch");
   return LBSA_OK;

@@ -81,9 +81,30 @@ cudaError_t launch_score_exact_f32(const float* q, const float* k, const lbsa_qk
 
 // block-mean proxy (meanpool.cu); workspace holds 2*B*H*nB*d floats + partials
 // nQ: rows of the score matrix, nB (query-block means) or n_valid (query tokens)
+// Per-token proxy logits on the tensor cores (token_logits_tc.cu).
+struct TokenLogitsArgs {
+  int G, H, nQ, nB, d;
+  float scale;            // 1 / sqrt(d)
+  float* scores;          // [G][nQ][nB] fp32 logits out
+  float2* part;           // [G][token_logits_parts(nQ, nB)] (max, sum of exp) per 32 tokens and 128 key blocks
+  int32_t* status;
+  long long wait_limit;
+};
+int token_logits_parts(int nQ, int nB);
+// hi / lo bf16 terms of n fp32 block means into out[0 .. n) and out[n .. 2n)
+cudaError_t launch_split_means(const float* kbar, long long n, void* out, cudaStream_t s);
+// tq: bf16 Q as lbsa_attend's Q map (box 64 x 128); tkb: the hi / lo terms as a 4D
+// bf16 map (d, nB, G, 2) with box 64 x 128 x 1 x 1, 128-byte swizzle
+cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const TokenLogitsArgs& a,
+                                     cudaStream_t s);
 size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ);
+// where, in the mean-pool workspace, the per-token path keeps the bf16 hi / lo
+// terms of the key-block means (2 x G x nB x d bf16)
+void* meanpool_split_ptr(void* ws);
+// tq / tkb: non-NULL for bf16 per-token mode, which then takes the tensor-core logits
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
-                            float* scores, void* workspace, cudaStream_t s);
+                            float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq = nullptr,
+                            const CUtensorMap* tkb = nullptr, int32_t* status = nullptr, long long wait_limit = 0);
 
 // selection (select.cu)
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,

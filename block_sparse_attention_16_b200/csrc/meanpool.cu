@@ -409,7 +409,8 @@ void launch_mean(const void* q, const void* k, const lbsa_qkv_desc& d, int block
 
 template <int D>
 cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens, float* scores,
-                void* ws, cudaStream_t s) {
+                void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb, int32_t* status,
+                long long wait_limit) {
   const long long G = static_cast<long long>(d.B) * d.H;
   float* qbar = static_cast<float*>(ws);
   float* kbar = qbar + G * nB * D;
@@ -430,6 +431,22 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
   }
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const dim3 lgrid(nTk, nTq, static_cast<unsigned>(G));
+  const long long n = static_cast<long long>(nQ) * nB;
+  const int chunks = static_cast<int>(std::min<long long>(tokens ? 256 : 64, (n + 2047) / 2048));
+  if (tokens && tq && tkb) {
+    // bf16 token rows: the logits on the tensor cores, from the means' hi / lo terms
+    // (written over the query-block means' slot, which this mode does not use)
+    cudaError_t e = launch_split_means(kbar, G * nB * D, qbar, s);
+    if (e != cudaSuccess) return e;
+    const int np = token_logits_parts(nQ, nB);
+    TokenLogitsArgs a{static_cast<int>(G), d.H, nQ, nB, D, scale, scores, part, status, wait_limit};
+    e = launch_token_logits_bf16(tq, tkb, a, s);
+    if (e != cudaSuccess) return e;
+    float2* head = part + G * np;
+    combine_partials_kernel<<<static_cast<unsigned>(G), 256, 0, s>>>(part, np, head);
+    normalize_kernel<<<dim3(chunks, static_cast<unsigned>(G)), 256, 0, s>>>(scores, head, n, 1);
+    return cudaGetLastError();
+  }
   if (!tokens) {
     logits_kernel<D, float, false><<<lgrid, 128, 0, s>>>(qbar, 0, 0, 0, d.H, kbar, nQ, nB, scale, scores, part);
   } else if (d.dtype == LBSA_BF16) {
@@ -440,8 +457,6 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
     logits_kernel<D, float, true><<<lgrid, 128, 0, s>>>(static_cast<const float*>(q), d.stride_b, d.stride_h,
                                                          d.stride_n, d.H, kbar, nQ, nB, scale, scores, part);
   }
-  const long long n = static_cast<long long>(nQ) * nB;
-  const int chunks = static_cast<int>(std::min<long long>(tokens ? 256 : 64, (n + 2047) / 2048));
   if (tokens) {
     float2* head = part + G * nTq * nTk;
     combine_partials_kernel<<<static_cast<unsigned>(G), 256, 0, s>>>(part, nTq * nTk, head);
@@ -457,13 +472,17 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
 size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
   const size_t nTk = (nB + kTk - 1) / kTk, nTq = (nQ + kTq - 1) / kTq;
-  return 2 * G * nB * d * sizeof(float) + (G * nTq * nTk + G) * sizeof(float2) + 256;
+  const size_t parts = std::max<size_t>(nTq * nTk, static_cast<size_t>(token_logits_parts(nQ, nB)));
+  return 2 * G * nB * d * sizeof(float) + (G * parts + G) * sizeof(float2) + 256;
 }
 
+void* meanpool_split_ptr(void* ws) { return ws; }   // the query-block means' slot: G x nB x d fp32
+
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
-                            float* scores, void* ws, cudaStream_t s) {
-  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s)
-                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s);
+                            float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb,
+                            int32_t* status, long long wait_limit) {
+  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit)
+                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit);
 }
 
 }  // namespace lbsa

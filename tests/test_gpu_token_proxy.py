@@ -87,6 +87,24 @@ def test_token_proxy_pipeline_matches_oracle(case):
     assert np.all(host(out)[empty] == 0)
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_token_scores_over_several_chunks(d):
+    """Tensor-core logits (bf16 token rows): 8,261 tokens (65 tiles of 128, the
+    last 69 rows), nB = 130 key blocks (two chunks of 128, the second with 2
+    valid columns; rows not a multiple of 4 floats): every score against the
+    fp64 oracle, and the head-scope selection on them bit-exact."""
+    wl = small_workload(f"tokchunks{d}", 1, 2, d, (11, 751, 1), 64, dtype="bf16", wid=330 + d)
+    assert wl.n_blocks == 130
+    q, k = (x.cuda() for x in make_qkv(wl)[:2])
+    scores = lbsa.lbsa_score(q, k, 64, mode="meanpool_token")
+    bs = lbsa.lbsa_select_tokens(scores, 64, TAU)
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_device_status() == 0 and lbsa.lbsa_get_status(bs) == 0
+    sc = host(scores)
+    assert_scores_close(sc, oracle.token_meanpool_scores(host(q), host(k), wl.n_valid, 64))
+    assert_csr_equal(token_csr(bs, wl.n_valid), oracle.select_contract(sc, TAU, "head"))
+
+
 def test_token_proxy_p1_keeps_every_pair_and_is_dense():
     wl = small_workload("tokdense", 1, 2, 128, (3, 8, 12), 64, dtype="bf16", wid=320)
     q, k, v = (x.cuda() for x in make_qkv(wl))
