@@ -127,6 +127,21 @@ int make_tmap_4d(CUtensorMap* map, const void* ptr, long long n0, long long n1, 
   return LBSA_OK;
 }
 
+// A dense fp32 [n2][n1][n0] array as a 3D tensor map with box 32 x box_rows x 1
+// (one 128-byte swizzle line a box row); n0 * 4 must be a multiple of 16.
+int make_tmap_f32_3d(CUtensorMap* map, void* ptr, long long n0, long long n1, long long n2, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(n0), static_cast<cuuint64_t>(n1), static_cast<cuuint64_t>(n2)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(n0) * 4, static_cast<cuuint64_t>(n0 * n1) * 4};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return LBSA_OK;
+}
+
 // Per-device state: a status word for calls without a blockset, and a memory
 // pool that serves blocksets and per-call scratch stream-ordered
 // (cudaMallocFromPoolAsync / cudaFreeAsync).  The pool keeps freed memory
@@ -283,8 +298,12 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
       if ((rc = make_tmap(&tq, q, desc, 128)) != LBSA_OK) return rc;
       const long long G = static_cast<long long>(desc->B) * desc->H;
       if ((rc = make_tmap_4d(&tkb, lbsa::meanpool_split_ptr(ws.ptr), desc->d, nB, G, 2, 128)) != LBSA_OK) return rc;
+      // the logits leave through TMA stores when a score row is a whole number of 16-byte units
+      CUtensorMap ts;
+      const bool tma_out = (nB % 4) == 0;
+      if (tma_out && (rc = make_tmap_f32_3d(&ts, scores, nB, nQ, G, 128)) != LBSA_OK) return rc;
       e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s, &tq, &tkb, ds->status,
-                                wait_limit());
+                                wait_limit(), tma_out ? &ts : nullptr);
     } else {
       e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s);
     }

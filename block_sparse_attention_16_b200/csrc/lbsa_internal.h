@@ -95,8 +95,10 @@ int token_logits_parts(int nQ, int nB);
 cudaError_t launch_split_means(const float* kbar, long long n, void* out, cudaStream_t s);
 // tq: bf16 Q as lbsa_attend's Q map (box 64 x 128); tkb: the hi / lo terms as a 4D
 // bf16 map (d, nB, G, 2) with box 64 x 128 x 1 x 1, 128-byte swizzle
-cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const TokenLogitsArgs& a,
-                                     cudaStream_t s);
+// ts: the logits [G][nQ][nB] as a 3D fp32 map (nB, nQ, G), box 32 x 128 x 1, or NULL
+// (direct stores; required when nB is not a multiple of 4)
+cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const CUtensorMap* ts,
+                                     const TokenLogitsArgs& a, cudaStream_t s);
 size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ);
 // where, in the mean-pool workspace, the per-token path keeps the bf16 hi / lo
 // terms of the key-block means (2 x G x nB x d bf16)
@@ -104,7 +106,8 @@ void* meanpool_split_ptr(void* ws);
 // tq / tkb: non-NULL for bf16 per-token mode, which then takes the tensor-core logits
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
                             float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq = nullptr,
-                            const CUtensorMap* tkb = nullptr, int32_t* status = nullptr, long long wait_limit = 0);
+                            const CUtensorMap* tkb = nullptr, int32_t* status = nullptr, long long wait_limit = 0,
+                            const CUtensorMap* ts = nullptr);
 
 // selection (select.cu)
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,

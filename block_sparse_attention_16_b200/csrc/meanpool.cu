@@ -410,7 +410,7 @@ void launch_mean(const void* q, const void* k, const lbsa_qkv_desc& d, int block
 template <int D>
 cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens, float* scores,
                 void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb, int32_t* status,
-                long long wait_limit) {
+                long long wait_limit, const CUtensorMap* ts) {
   const long long G = static_cast<long long>(d.B) * d.H;
   float* qbar = static_cast<float*>(ws);
   float* kbar = qbar + G * nB * D;
@@ -440,7 +440,7 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
     if (e != cudaSuccess) return e;
     const int np = token_logits_parts(nQ, nB);
     TokenLogitsArgs a{static_cast<int>(G), d.H, nQ, nB, D, scale, scores, part, status, wait_limit};
-    e = launch_token_logits_bf16(tq, tkb, a, s);
+    e = launch_token_logits_bf16(tq, tkb, ts, a, s);
     if (e != cudaSuccess) return e;
     float2* head = part + G * np;
     combine_partials_kernel<<<static_cast<unsigned>(G), 256, 0, s>>>(part, np, head);
@@ -480,9 +480,9 @@ void* meanpool_split_ptr(void* ws) { return ws; }   // the query-block means' sl
 
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
                             float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb,
-                            int32_t* status, long long wait_limit) {
-  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit)
-                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit);
+                            int32_t* status, long long wait_limit, const CUtensorMap* ts) {
+  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts)
+                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts);
 }
 
 }  // namespace lbsa

@@ -41,17 +41,19 @@ struct TLLayout {
   static constexpr int TILE_BYTES = kCols * D * 2;        // one term (hi or lo) of one chunk
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = Q_BYTES;                 // [stage][term] tiles
-  static constexpr int OFF_BAR = OFF_RING + 4 * TILE_BYTES;
+  static constexpr int OFF_OUT = OFF_RING + 4 * TILE_BYTES;  // two 128 x 32 fp32 store boxes (16 KB each)
+  static constexpr int OUT_BYTES = kRows * 32 * 4;
+  static constexpr int OFF_BAR = OFF_OUT + 2 * OUT_BYTES;
   // q_full, q_empty, kv_full[2], kv_empty[2], acc_full[2], acc_empty[2], drain
   static constexpr int NBAR = 11;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // [0] tmem base [1] abort
   static constexpr int BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 };
 
-template <int D>
+template <int D, bool TMA_OUT>
 __global__ void __launch_bounds__(kTLThreads, 1)
 token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kb,
-                       const TokenLogitsArgs args) {
+                       const __grid_constant__ CUtensorMap tmap_s, const TokenLogitsArgs args) {
   using L = TLLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,6 +171,7 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     // ------------------------------------------------------------ epilogue (warps 0-3)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     long long step = 0;
+    long long boxes = 0;                     // TMA store boxes issued (alternating staging buffers)
     bool ok = true;
     for (long long item = blockIdx.x; ok && item < items; item += gridDim.x) {
       const int g = static_cast<int>(item / nTq), tq = static_cast<int>(item % nTq);
@@ -177,7 +180,8 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
       float* srow = args.scores + (static_cast<long long>(g) * args.nQ + (rvalid ? row : 0)) * args.nB;
       for (int c = 0; c < nC; ++c, ++step) {
         const int st = static_cast<int>(step & 1);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(acc_full + st, (step >> 1) & 1, wl, args.status, abort_flag))))
+        // the four warps decide together (they share named barriers below)
+        if (!(ok = named_bar_and(2, 128, mbar_wait(acc_full + st, (step >> 1) & 1, wl, args.status, abort_flag))))
           break;
         tc_fence_after();
         uint32_t v[128];
@@ -196,26 +200,43 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
           v[j] = __float_as_uint(x);
           if (rvalid && j < ncol) mx = fmaxf(mx, x);
         }
-        if (rvalid) {
-          float* dst = srow + col0;
-          if (ncol == kCols && (args.nB & 3) == 0) {
+        if (TMA_OUT) {
+          // four 128 x 32 boxes through two swizzled staging buffers: row t's
+          // 16-byte unit u sits at unit u ^ (t & 7) of its 128-byte line; one
+          // thread issues each TMA store (clipped at nQ rows and nB columns)
+          const int t = warp * 32 + lane;
 #pragma unroll
-            for (int j = 0; j < 128; j += 4)
-              *reinterpret_cast<float4*>(dst + j) = make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                                                __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-          } else {
+          for (int k = 0; k < 4; ++k, ++boxes) {
+            uint8_t* box = smem + L::OFF_OUT + (boxes & 1) * L::OUT_BYTES;
+            if (boxes >= 2) {
+              if (t == 0) tma_store_wait_read<1>();       // the store that last read this box is done with it
+              named_bar_sync(1, 128);
+            }
 #pragma unroll
-            for (int j = 0; j < 128; ++j)
-              if (j < ncol) dst[j] = __uint_as_float(v[j]);
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(box + t * 128 + ((u ^ (t & 7)) << 4)) =
+                  make_uint4(v[32 * k + 4 * u], v[32 * k + 4 * u + 1], v[32 * k + 4 * u + 2], v[32 * k + 4 * u + 3]);
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (t == 0) {
+              tma_store_3d(&tmap_s, box, col0 + 32 * k, tq * kRows, g);
+              tma_store_commit();
+            }
           }
+        } else if (rvalid) {
+          float* dst = srow + col0;
+#pragma unroll
+          for (int j = 0; j < 128; ++j)
+            if (j < ncol) dst[j] = __uint_as_float(v[j]);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float sm = 0.f;
         if (rvalid && mx != -INFINITY) {
+          const float mxl = mx * 1.4426950408889634f;
 #pragma unroll
           for (int j = 0; j < 128; ++j)
-            if (j < ncol) sm += expf(__uint_as_float(v[j]) - mx);
+            if (j < ncol) sm += ex2(fmaf(__uint_as_float(v[j]), 1.4426950408889634f, -mxl));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
@@ -223,6 +244,7 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
           args.part[((static_cast<long long>(g) * nTq + tq) * nC + c) * 4 + warp] = make_float2(mx, sm);
       }
     }
+    if (TMA_OUT && warp == 0 && lane == 0) tma_store_wait<0>();   // the logits are in global memory
   }
   tc_fence_before();
   __syncthreads();
@@ -264,19 +286,22 @@ cudaError_t launch_split_means(const float* kbar, long long n, void* out, cudaSt
   return cudaGetLastError();
 }
 
-cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const TokenLogitsArgs& a,
-                                     cudaStream_t s) {
+cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const CUtensorMap* ts,
+                                     const TokenLogitsArgs& a, cudaStream_t s) {
   if (!(a.d == 64 || a.d == 128) || a.nB < 1 || a.nQ < 1 || a.G < 1) return cudaErrorInvalidValue;
   const long long items = static_cast<long long>(a.G) * ((a.nQ + kRows - 1) / kRows);
   const unsigned grid = static_cast<unsigned>(std::min<long long>(items, tl_sms()));
   auto go = [&](auto kern, int smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTLThreads, smem, s>>>(*tq, *tkb, a);
+    kern<<<grid, kTLThreads, smem, s>>>(*tq, *tkb, ts ? *ts : *tq, a);
     return cudaGetLastError();
   };
-  return a.d == 128 ? go(token_logits_tc_kernel<128>, TLLayout<128>::BYTES)
-                    : go(token_logits_tc_kernel<64>, TLLayout<64>::BYTES);
+  if (ts)
+    return a.d == 128 ? go(token_logits_tc_kernel<128, true>, TLLayout<128>::BYTES)
+                      : go(token_logits_tc_kernel<64, true>, TLLayout<64>::BYTES);
+  return a.d == 128 ? go(token_logits_tc_kernel<128, false>, TLLayout<128>::BYTES)
+                    : go(token_logits_tc_kernel<64, false>, TLLayout<64>::BYTES);
 }
 
 }  // namespace lbsa
