@@ -354,7 +354,8 @@ struct HeadState {
 
 constexpr int kDigitBits = 10;
 constexpr int kBins = 1 << kDigitBits;
-constexpr long long kHistPerCta = 4096;     // elements per histogram CTA (256 threads x 16)
+constexpr long long kHistPerCta = 16384;    // most elements a histogram CTA sees (256 threads x 64)
+constexpr int kLoBits = 18;                  // weight split for the 32-bit shared sums (see head_hist_kernel)
 
 // After pass k, run by the last histogram CTA of the head (256 threads, bins
 // 4t .. 4t+3 per thread): pick the digit where the weight at or above crosses
@@ -438,8 +439,9 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
                                                         unsigned long long* __restrict__ hist,
                                                         HeadState* __restrict__ st, int32_t* __restrict__ status) {
   __shared__ int is_last;
-  // weights split into 20 low and 13 high bits, summed with 32-bit shared
-  // atomics (a CTA sees at most kHistPerCta elements: the low sums stay < 2^32)
+  // weights (< 2^33) split into 18 low and 15 high bits, summed with 32-bit
+  // shared atomics: a CTA sees at most kHistPerCta = 2^14 elements, so the low
+  // sums stay below 2^32 and the high ones below 2^29
   __shared__ uint32_t sh_lo[kBins], sh_hi[kBins];
   __shared__ unsigned int smax;
   __shared__ int sbad;
@@ -460,8 +462,8 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
   const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + static_cast<long long>(g) * seg_len;
   unsigned int lmax = 0;
   int lbad = 0;
-  // a thread's elements (16 at the launch's grid of one CTA per kHistPerCta)
-  // are all loaded before any is binned, so their DRAM round trips overlap
+  // a thread's elements come in batches of 16, all loaded before any is
+  // binned, so their DRAM round trips overlap
   constexpr int kBatch = 16;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < seg_len;
@@ -485,8 +487,8 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
       const uint64_t w = fixed_weight(b);
       if (w) {
         const uint32_t bin = (b >> shift) & (kBins - 1);
-        atomicAdd(&sh_lo[bin], static_cast<uint32_t>(w & 0xFFFFFull));
-        atomicAdd(&sh_hi[bin], static_cast<uint32_t>(w >> 20));
+        atomicAdd(&sh_lo[bin], static_cast<uint32_t>(w & ((1ull << kLoBits) - 1)));
+        atomicAdd(&sh_hi[bin], static_cast<uint32_t>(w >> kLoBits));
       }
     }
   }
@@ -497,7 +499,7 @@ __global__ void __launch_bounds__(256) head_hist_kernel(const float* __restrict_
   __syncthreads();
   unsigned long long* gh = hist + static_cast<long long>(g) * kBins;
   for (int i = threadIdx.x; i < kBins; i += blockDim.x) {
-    const unsigned long long v = (static_cast<unsigned long long>(sh_hi[i]) << 20) + sh_lo[i];
+    const unsigned long long v = (static_cast<unsigned long long>(sh_hi[i]) << kLoBits) + sh_lo[i];
     if (v) atomicAdd(gh + i, v);
   }
   if (threadIdx.x == 0 && pass == 0) {
@@ -622,16 +624,28 @@ __global__ void __launch_bounds__(256) token_emit_kernel(const float* __restrict
     }
     const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + (static_cast<long long>(g) * nQ + r) * nB;
     uint32_t ties_before = all ? 0u : static_cast<uint32_t>(tiebase[static_cast<long long>(g) * nQ + r]);
-    for (int j0 = 0; j0 < nB; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t b = (j < nB) ? __ldg(x + j) : 0u;
-      const bool tie = (j < nB) && b == tb;
-      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
-      const uint32_t rank = ties_before + __popc(tmask & lt_mask);
-      const bool k = (j < nB) && (all || b > tb || (tie && rank < need));
-      const uint32_t kmask = __ballot_sync(0xffffffffu, k);
-      if (lane == 0) keep[tt][j0 >> 5] = kmask;
-      ties_before += __popc(tmask);
+    // eight 32-column loads in flight before the first is used
+    for (int j1 = 0; j1 < nB; j1 += 256) {
+      uint32_t bv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j1 + 32 * u + lane;
+        bv[u] = (j < nB) ? __ldg(x + j) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j0 = j1 + 32 * u;
+        if (j0 >= nB) break;
+        const int j = j0 + lane;
+        const uint32_t b = bv[u];
+        const bool tie = (j < nB) && b == tb;
+        const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+        const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+        const bool k = (j < nB) && (all || b > tb || (tie && rank < need));
+        const uint32_t kmask = __ballot_sync(0xffffffffu, k);
+        if (lane == 0) keep[tt][j0 >> 5] = kmask;
+        ties_before += __popc(tmask);
+      }
     }
   }
   __syncthreads();
@@ -1198,6 +1212,22 @@ cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, i
   return cudaGetLastError();
 }
 
+// Histogram CTAs per head: at most kHistPerCta elements each (the 32-bit shared
+// sums rely on that bound); fewer per CTA, down to 4,096, while the launch would
+// otherwise hold fewer than four CTAs per SM.
+static long long hist_chunks(long long seg, int G) {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  long long per = kHistPerCta;
+  while (per > 4096 && static_cast<long long>(G) * ((seg + per - 1) / per) < 4ll * sms) per >>= 1;
+  return (seg + per - 1) / per;
+}
+
 size_t select_head_workspace_bytes(int B, int H, int nB, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
   if (nQ <= 0) nQ = nB;
@@ -1216,7 +1246,7 @@ cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double
   if (e != cudaSuccess) return e;
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
+  const int chunks = static_cast<int>(hist_chunks(seg, G));
   for (int pass = 0; pass < 3; ++pass) {
     head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, P, keep_all, hist, st, bs->status);
   }
@@ -1241,8 +1271,7 @@ cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int 
   if (e != cudaSuccess) return e;
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  // one histogram CTA per kHistPerCta pairs (its 32-bit shared sums rely on that bound)
-  const long long chunks = (seg + kHistPerCta - 1) / kHistPerCta;
+  const long long chunks = hist_chunks(seg, G);
   if (chunks > 65535) return cudaErrorInvalidValue;
   const unsigned hc = static_cast<unsigned>(chunks);
   for (int pass = 0; pass < 3; ++pass) {
@@ -1382,7 +1411,7 @@ extern "C" int lbsa_select_head_noalloc(const float* scores, int32_t B, int32_t 
   if (e != cudaSuccess) return set_error(LBSA_ERR_CUDA, cudaGetErrorString(e));
   const uint32_t P = fixed_p(p);
   const int keep_all = p >= 1.0 ? 1 : 0;
-  const int chunks = static_cast<int>((seg + kHistPerCta - 1) / kHistPerCta);
+  const int chunks = static_cast<int>(hist_chunks(seg, G));
   for (int pass = 0; pass < 3; ++pass) {
     head_hist_kernel<<<dim3(chunks, G), 256, 0, s>>>(scores, seg, pass, P, keep_all, hist, st, status);
   }
