@@ -372,7 +372,8 @@ int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t b
     DeviceState* ds = nullptr;
     Scratch ws;
     if ((rc = device_state(&ds)) != LBSA_OK ||
-        (rc = scratch_alloc(ds, lbsa::select_head_workspace_bytes(B, H, nB), s, &ws)) != LBSA_OK) {
+        (!lbsa::select_head_one_launch(nB) &&
+         (rc = scratch_alloc(ds, lbsa::select_head_workspace_bytes(B, H, nB), s, &ws)) != LBSA_OK)) {
       lbsa_free(bs);
       return rc;
     }

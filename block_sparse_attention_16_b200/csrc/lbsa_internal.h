@@ -118,6 +118,9 @@ cudaError_t launch_head_floor(const int32_t* counts, int G, int nB, int block, i
                               cudaStream_t s);
 // nQ: rows of each head's pairs (nB query blocks, or n_valid query tokens); 0 means nB
 size_t select_head_workspace_bytes(int B, int H, int nB, int nQ = 0);
+// block-scope head selection runs as one cluster launch without workspace for
+// heads whose nB x nB scores fit the cluster's shared memory
+bool select_head_one_launch(int nB);
 cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs,
                                void* workspace, cudaStream_t s);
 // per-token scope: nQ = n_valid token rows of nB key blocks, 64-token blocks; writes

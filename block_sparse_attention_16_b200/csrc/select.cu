@@ -16,6 +16,7 @@
 // still reaches T.  Every element above tb is kept; of the elements equal to
 // tb (all of weight w(tb)), the ceil((T - S(tb+1)) / w(tb)) with the lowest
 // flat indices are kept.  This is exactly the sorted-prefix rule.
+#include <cooperative_groups.h>
 #include <cstdio>
 #include <mutex>
 
@@ -592,6 +593,278 @@ __global__ void head_emit_kernel(const float* __restrict__ scores, int G, int nB
     ties_before += __popc(tmask);
   }
   if (lane == 0) counts[row] = base;
+}
+
+// Head scope in one launch, for segments that fit the cluster's shared memory:
+// a cluster of kHC CTAs per (batch, head) segment of nQ x nB scores (rows of
+// nB; flat index i*nB + j).  CTA r owns rows [r*rpc, (r+1)*rpc), rpc =
+// ceil(nQ / kHC), and keeps them in shared memory after the first pass.  Each
+// of the three 10-bit digit passes builds the CTA's exact histogram of
+// fixed-point weights (16/17-bit split 32-bit shared atomics, folded into
+// 64-bit bins every 2^15 scores, so the 32-bit sums stay exact); the cluster
+// sums the bins through distributed shared memory (CTA r reduces bins
+// [128r, 128r + 128)) and every CTA takes the same digit decision from the
+// same sums.  Ties (scores equal to the threshold value) are ranked in flat
+// order from per-row counts and the CTAs' totals; then each warp emits rows.
+// All control flow that spans cluster barriers is uniform over the cluster.
+constexpr int kHC = 8;
+constexpr int kHCT = 512;                     // threads a CTA
+constexpr int kHCMaxRows = 2 * kHCT;          // rows a CTA can own
+constexpr int kHCMaxSlice = 40960;            // scores a CTA keeps in shared memory (160 KB)
+
+// S[i] = weight of bins >= 2t + i over the CTA's 1024 bins (kHCT threads x 2)
+__device__ __forceinline__ void hc_suffix(const unsigned long long (&v)[2], unsigned long long (&S)[3],
+                                          unsigned long long* warp_tot) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  unsigned long long x = v[0] + v[1];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
+    if (lane + o < 32) x += y;
+  }
+  if (lane == 0) warp_tot[w] = x;
+  __syncthreads();
+  unsigned long long later = 0;
+  for (int u = w + 1; u < kHCT / 32; ++u) later += warp_tot[u];
+  S[0] = x + later;
+  S[1] = S[0] - v[0];
+  S[2] = S[1] - v[1];
+  __syncthreads();                            // warp_tot is reused by the next call
+}
+
+__global__ void __cluster_dims__(kHC, 1, 1) __launch_bounds__(kHCT)
+head_select_cluster_kernel(const float* __restrict__ scores, int nQ, int nB, uint32_t Pfix, int keep_all_p,
+                           int32_t* __restrict__ counts, int32_t* __restrict__ cols, int32_t* __restrict__ status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  extern __shared__ __align__(16) uint32_t slice[];   // this CTA's rows, [row][nB] score bits
+  __shared__ uint32_t h_lo[kBins], h_hi[kBins];
+  __shared__ unsigned long long h64[kBins];    // this CTA's histogram of the pass
+  __shared__ unsigned long long red[kBins / kHC];   // bins [r*128, r*128 + 128) summed over the cluster
+  __shared__ unsigned long long warp_tot[kHCT / 32];
+  __shared__ int tiecnt[kHCMaxRows];
+  __shared__ unsigned int s_max, s_ties;
+  __shared__ int s_bad;
+  __shared__ unsigned long long s_state[2];    // T, above
+  __shared__ unsigned int s_dec[4];            // prefix, tb, need, mode (0 search, 1 resolved, 2 keep all)
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int r = static_cast<int>(cl.block_rank());
+  const long long g = blockIdx.x / kHC;
+  const int rpc = (nQ + kHC - 1) / kHC;
+  const int r0 = min(nQ, r * rpc), r1 = min(nQ, r0 + rpc);
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + (g * nQ + r0) * static_cast<long long>(nB);
+  const int n = (r1 - r0) * nB;                // this CTA's scores (<= kHCMaxSlice)
+  if (t == 0) {
+    s_max = 0;
+    s_bad = 0;
+    s_dec[0] = 0;
+    s_dec[3] = keep_all_p ? 2u : 0u;
+    s_state[1] = 0;
+  }
+  __syncthreads();
+  for (int pass = 0; pass < 3; ++pass) {
+    const bool search = s_dec[3] == 0 || pass == 0;   // uniform: every CTA holds the same decision
+    if (search) {
+      const int shift = 20 - kDigitBits * pass;
+      const unsigned int prefix = s_dec[0];
+      for (int i = t; i < kBins; i += kHCT) {
+        h_lo[i] = 0u;
+        h_hi[i] = 0u;
+        h64[i] = 0ull;
+      }
+      __syncthreads();
+      unsigned int lmax = 0;
+      int lbad = 0;
+      auto bin_one = [&](uint32_t b) {
+        if (b >= kInvalidBits) {
+          lbad = 1;
+          return;
+        }
+        if (pass == 0) lmax = max(lmax, b);
+        if (pass > 0 && (b >> (shift + kDigitBits)) != prefix) return;
+        const uint64_t w = fixed_weight(b);
+        if (w) {
+          const uint32_t bin = (b >> shift) & (kBins - 1);
+          atomicAdd(&h_lo[bin], static_cast<uint32_t>(w & 0xFFFFull));
+          atomicAdd(&h_hi[bin], static_cast<uint32_t>(w >> 16));
+        }
+      };
+      // rounds of at most 2^15 scores: 16-bit low parts sum below 2^31, 17-bit high parts below 2^32
+      for (int q0 = 0; q0 < n; q0 += 32768) {
+        const int q1 = min(n, q0 + 32768);
+        if (pass == 0) {
+          // from global memory (16-byte loads when rows are whole 16-byte units), kept in shared memory
+          if ((nB & 3) == 0) {
+            for (int i0 = q0 + 4 * t; i0 < q1; i0 += 4 * kHCT * 4) {
+              uint4 v[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                v[u] = (i0 + 4 * kHCT * u < q1) ? __ldg(reinterpret_cast<const uint4*>(x + i0 + 4 * kHCT * u))
+                                                 : make_uint4(0, 0, 0, 0);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int i = i0 + 4 * kHCT * u;
+                if (i >= q1) break;
+                *reinterpret_cast<uint4*>(slice + i) = v[u];
+                bin_one(v[u].x);
+                bin_one(v[u].y);
+                bin_one(v[u].z);
+                bin_one(v[u].w);
+              }
+            }
+          } else {
+            for (int i = q0 + t; i < q1; i += kHCT) {
+              const uint32_t b = __ldg(x + i);
+              slice[i] = b;
+              bin_one(b);
+            }
+          }
+        } else {
+          for (int i = q0 + t; i < q1; i += kHCT) bin_one(slice[i]);
+        }
+        __syncthreads();
+        for (int i = t; i < kBins; i += kHCT) {
+          h64[i] += (static_cast<unsigned long long>(h_hi[i]) << 16) + h_lo[i];
+          h_lo[i] = 0u;
+          h_hi[i] = 0u;
+        }
+        __syncthreads();
+      }
+      if (pass == 0) {
+        atomicMax(&s_max, lmax);
+        if (lbad) atomicOr(&s_bad, 1);
+      }
+    }
+    cl.sync();                                 // every CTA's h64, s_max, s_bad are final
+    if (search) {
+      if (t < kBins / kHC) {
+        unsigned long long acc = 0;
+        for (int q = 0; q < kHC; ++q) acc += cl.map_shared_rank(h64, q)[r * (kBins / kHC) + t];
+        red[t] = acc;
+      }
+      if (pass == 0 && t == kHCT - 1) {
+        unsigned int mx = 0;
+        int bad = 0;
+        for (int q = 0; q < kHC; ++q) {
+          mx = max(mx, *cl.map_shared_rank(&s_max, q));
+          bad |= *cl.map_shared_rank(&s_bad, q);
+        }
+        s_dec[1] = mx;                         // the threshold value if T turns out 0
+        s_dec[2] = static_cast<unsigned int>(bad);
+      }
+    }
+    cl.sync();                                 // every CTA's red is final
+    if (search) {
+      unsigned long long v[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int b = 2 * t + i;
+        v[i] = cl.map_shared_rank(red, b / (kBins / kHC))[b % (kBins / kHC)];
+      }
+      unsigned long long S[3];
+      hc_suffix(v, S, warp_tot);               // (its barriers also publish s_dec[1..2])
+      if (pass == 0 && t == 0) {
+        if (s_dec[2]) {
+          if (r == 0) raise_status(status, LBSA_ERR_INVALID_SCORES);
+          s_dec[3] = 2u;
+        } else if (s_dec[3] != 2u) {
+          s_state[0] = threshold_T(S[0], Pfix);
+          s_state[1] = 0;
+          if (s_state[0] == 0) {
+            s_dec[2] = 1u;                     // keep one: the highest score (tb = the max), lowest index
+            s_dec[3] = 1u;
+          }
+        }
+      }
+      __syncthreads();
+      if (s_dec[3] == 0) {
+        const unsigned long long T = s_state[0], above = s_state[1];
+        const unsigned int prefix = s_dec[0];
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          if (above + S[i] >= T && above + S[i + 1] < T) {
+            const unsigned int b = static_cast<unsigned int>(2 * t + i);
+            s_state[1] = above + S[i + 1];
+            s_dec[0] = (prefix << kDigitBits) | b;
+            if (pass == 2) {
+              const unsigned int tb = (prefix << kDigitBits) | b;
+              const unsigned long long ww = fixed_weight(tb);
+              s_dec[1] = tb;
+              s_dec[2] = static_cast<unsigned int>((T - (above + S[i + 1]) + ww - 1) / ww);
+              s_dec[3] = 1u;
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const bool all = s_dec[3] == 2u;
+  const uint32_t tb = s_dec[1], need = s_dec[2];
+  // ties per row of this CTA, the CTA's total, and the cluster's totals before it
+  if (t == 0) s_ties = 0;
+  __syncthreads();
+  for (int i = warp; i < r1 - r0; i += kHCT / 32) {
+    int c = 0;
+    if (!all)
+      for (int j = lane; j < nB; j += 32) c += (slice[i * nB + j] == tb);
+    c = __reduce_add_sync(0xffffffffu, static_cast<unsigned>(c));
+    if (lane == 0) {
+      tiecnt[i] = c;
+      atomicAdd(&s_ties, static_cast<unsigned>(c));
+    }
+  }
+  __syncthreads();
+  cl.sync();
+  unsigned int base = 0;
+  for (int q = 0; q < r; ++q) base += *cl.map_shared_rank(&s_ties, q);
+  cl.sync();                                   // no CTA leaves while another reads its total
+  {
+    // exclusive scan of the rows' tie counts (at most kHCMaxRows = 2 x kHCT rows)
+    const int nr = r1 - r0;
+    const int a = (2 * t < nr) ? tiecnt[2 * t] : 0, b = (2 * t + 1 < nr) ? tiecnt[2 * t + 1] : 0;
+    unsigned int incl = static_cast<unsigned int>(a + b);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    unsigned int before = base + incl - static_cast<unsigned int>(a + b);
+    for (int u = 0; u < warp; ++u) before += static_cast<unsigned int>(warp_tot[u]);
+    __syncthreads();
+    if (2 * t < nr) tiecnt[2 * t] = static_cast<int>(before);
+    if (2 * t + 1 < nr) tiecnt[2 * t + 1] = static_cast<int>(before + a);
+  }
+  __syncthreads();
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int i = warp; i < r1 - r0; i += kHCT / 32) {
+    const long long row = g * nQ + r0 + i;
+    int32_t* out = cols + row * nB;
+    if (all) {
+      for (int j = lane; j < nB; j += 32) out[j] = j;
+      if (lane == 0) counts[row] = nB;
+      continue;
+    }
+    const uint32_t* xr = slice + i * nB;
+    uint32_t ties_before = static_cast<uint32_t>(tiecnt[i]);
+    int cnt = 0;
+    for (int j0 = 0; j0 < nB; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t b = (j < nB) ? xr[j] : 0u;
+      const bool tie = (j < nB) && b == tb;
+      const uint32_t tmask = __ballot_sync(0xffffffffu, tie);
+      const uint32_t rank = ties_before + __popc(tmask & lt_mask);
+      const bool keep = (j < nB) && (b > tb || (tie && rank < need));
+      const uint32_t kmask = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[cnt + __popc(kmask & lt_mask)] = j;
+      cnt += __popc(kmask);
+      ties_before += __popc(tmask);
+    }
+    if (lane == 0) counts[row] = cnt;
+  }
 }
 
 // Per-token scope: emit, for each query block, the key blocks kept by at
@@ -1228,6 +1501,10 @@ static long long hist_chunks(long long seg, int G) {
   return (seg + per - 1) / per;
 }
 
+bool select_head_one_launch(int nB) {
+  return static_cast<long long>((nB + kHC - 1) / kHC) * nB <= kHCMaxSlice;
+}
+
 size_t select_head_workspace_bytes(int B, int H, int nB, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
   if (nQ <= 0) nQ = nB;
@@ -1237,6 +1514,17 @@ size_t select_head_workspace_bytes(int B, int H, int nB, int nQ) {
 cudaError_t launch_select_head(const float* scores, int B, int H, int nB, double p, lbsa_blockset* bs, void* ws,
                                cudaStream_t s) {
   const int G = B * H;
+  if (select_head_one_launch(nB)) {
+    const long long slice = static_cast<long long>((nB + kHC - 1) / kHC) * nB;
+    // one launch: a cluster of kHC CTAs per head, each keeping its rows in shared memory
+    const int smem = static_cast<int>(slice * sizeof(uint32_t));
+    cudaError_t e = cudaFuncSetAttribute(head_select_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    head_select_cluster_kernel<<<static_cast<unsigned>(G) * kHC, kHCT, smem, s>>>(scores, nB, nB, fixed_p(p),
+                                                                                 p >= 1.0 ? 1 : 0, bs->counts,
+                                                                                 bs->cols, bs->status);
+    return cudaGetLastError();
+  }
   const long long seg = static_cast<long long>(nB) * nB;
   unsigned long long* hist = reinterpret_cast<unsigned long long*>(ws);
   HeadState* st = reinterpret_cast<HeadState*>(hist + static_cast<size_t>(G) * kBins);
