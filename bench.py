@@ -386,9 +386,24 @@ def extra_measurements(lbsa, wl, dev, qp, kp, vp, perm, q, k, v, pk):
             o_ = lbsa.lbsa_attend(a_, b_, c_, x_)
             return lbsa.lbsa_permute([o_], pm, inverse=True)[0]
         prow[part] = _timer(call)["median"]
+    # the 3D call's stages, and the per-token proxy (every query token against the key-block means)
+    pm = lbsa.lbsa_partition_perm(T, H, W, "3d", device=dev)
+    a3, b3, c3 = lbsa.lbsa_permute([qq, kk, vv], pm)
+    s3 = lbsa.lbsa_score(a3, b3, wp.block, mode="meanpool")
+    x3 = lbsa.lbsa_select(s3, wp.block, wp.p, "head")
+    stages = {"score_ms": _timer(lambda: lbsa.lbsa_score(a3, b3, wp.block, mode="meanpool", scores=s3))["median"],
+              "select_ms": _timer(lambda: lbsa.lbsa_select(s3, wp.block, wp.p, "head"))["median"],
+              "attend_ms": _timer(lambda: lbsa.lbsa_attend(a3, b3, c3, x3))["median"]}
+    st3 = lbsa.lbsa_score(a3, b3, wp.block, mode="meanpool_token")
+    xt3 = lbsa.lbsa_select_tokens(st3, wp.block, wp.p)
+    token = {"score_ms": _timer(lambda: lbsa.lbsa_score(a3, b3, wp.block, mode="meanpool_token",
+                                                        scores=st3))["median"],
+             "select_ms": _timer(lambda: lbsa.lbsa_select_tokens(st3, wp.block, wp.p))["median"],
+             "attend_ms": _timer(lambda: lbsa.lbsa_attend(a3, b3, c3, xt3))["median"]}
     out["config3"] = {"workload": "mean-pooled proxy, head scope tau=0.25, Wan-like shape",
-                      "call_ms": prow, "call_ms_mean_of_cycle": sum(prow.values()) / 3}
-    del qq, kk, vv
+                      "call_ms": prow, "call_ms_mean_of_cycle": sum(prow.values()) / 3,
+                      "stages_3d_ms": stages, "per_token_3d_ms": token}
+    del qq, kk, vv, a3, b3, c3, s3, x3, st3, xt3
 
     # config 0: tiny fp32 case
     wt = get_workload("tiny")

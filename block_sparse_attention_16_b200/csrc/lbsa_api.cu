@@ -304,6 +304,17 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
       if (tma_out && (rc = make_tmap_f32_3d(&ts, scores, nB, nQ, G, 128)) != LBSA_OK) return rc;
       e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s, &tq, &tkb, ds->status,
                                 wait_limit(), tma_out ? &ts : nullptr);
+    } else if (!tokens && desc->dtype == LBSA_BF16 && nB % 4 == 0) {
+      // the block-mean logits on the tensor cores: both means as bf16 hi / lo terms
+      const long long G = static_cast<long long>(desc->B) * desc->H;
+      void *qs, *ks;
+      lbsa::meanpool_block_split_ptrs(ws.ptr, desc->B, desc->H, nB, desc->d, &qs, &ks);
+      CUtensorMap tqs, tks, ts;
+      if ((rc = make_tmap_4d(&tqs, qs, desc->d, nB, G, 2, 128)) != LBSA_OK) return rc;
+      if ((rc = make_tmap_4d(&tks, ks, desc->d, nB, G, 2, 128)) != LBSA_OK) return rc;
+      if ((rc = make_tmap_f32_3d(&ts, scores, nB, nB, G, 128)) != LBSA_OK) return rc;
+      e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s, nullptr, &tks, ds->status,
+                                wait_limit(), &ts, &tqs);
     } else {
       e = lbsa::launch_meanpool(q, k, *desc, block, nB, tokens, scores, ws.ptr, s);
     }

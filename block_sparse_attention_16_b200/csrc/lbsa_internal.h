@@ -89,25 +89,29 @@ struct TokenLogitsArgs {
   float2* part;           // [G][token_logits_parts(nQ, nB)] (max, sum of exp) per 32 tokens and 128 key blocks
   int32_t* status;
   long long wait_limit;
+  int cpi = 0;            // 128-column chunks a work item takes (set by the launcher)
 };
 int token_logits_parts(int nQ, int nB);
-// hi / lo bf16 terms of n fp32 block means into out[0 .. n) and out[n .. 2n)
-cudaError_t launch_split_means(const float* kbar, long long n, void* out, cudaStream_t s);
 // tq: bf16 Q as lbsa_attend's Q map (box 64 x 128); tkb: the hi / lo terms as a 4D
 // bf16 map (d, nB, G, 2) with box 64 x 128 x 1 x 1, 128-byte swizzle
 // ts: the logits [G][nQ][nB] as a 3D fp32 map (nB, nQ, G), box 32 x 128 x 1, or NULL
 // (direct stores; required when nB is not a multiple of 4)
+// q_split: tq is instead the query-block means' hi / lo terms as a 4D bf16 map
+// (d, nQ, G, 2) like tkb (the block-mean proxy); then ts must be given
 cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const CUtensorMap* ts,
-                                     const TokenLogitsArgs& a, cudaStream_t s);
+                                     const TokenLogitsArgs& a, cudaStream_t s, bool q_split = false);
 size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ);
 // where, in the mean-pool workspace, the per-token path keeps the bf16 hi / lo
 // terms of the key-block means (2 x G x nB x d bf16)
 void* meanpool_split_ptr(void* ws);
+// the block-mean proxy's hi / lo terms of the query-block and key-block means
+// (each 2 x G x nB x d bf16), after the fp32 means and the partials
+void meanpool_block_split_ptrs(void* ws, int B, int H, int nB, int d, void** qs, void** ks);
 // tq / tkb: non-NULL for bf16 per-token mode, which then takes the tensor-core logits
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
                             float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq = nullptr,
                             const CUtensorMap* tkb = nullptr, int32_t* status = nullptr, long long wait_limit = 0,
-                            const CUtensorMap* ts = nullptr);
+                            const CUtensorMap* ts = nullptr, const CUtensorMap* tqs = nullptr);
 
 // selection (select.cu)
 cudaError_t launch_select_row(const float* scores, int R, int nB, double p, lbsa_blockset* bs,

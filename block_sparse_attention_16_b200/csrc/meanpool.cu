@@ -70,11 +70,14 @@ struct Raw8<float> {
 // before the current item's sums are reduced, so DRAM traffic continues
 // through the reduction.  Reduction: lanes of a warp that share v by
 // shuffles, then the eight warps through double-buffered shared memory (one
-// barrier per item).
+// barrier per item).  qs / ks (optional): the means' bf16 hi / lo terms for the
+// tensor-core logits, hi = bf16(m) at [item*D + c], lo = bf16(m - hi) at n + that.
 template <typename T, int D, int MAXR>
 __global__ void __launch_bounds__(256) block_mean_kernel(const T* __restrict__ q, const T* __restrict__ k,
                                                          lbsa_qkv_desc desc, int block, int nB, long long items,
-                                                         float* __restrict__ qbar, float* __restrict__ kbar) {
+                                                         float* __restrict__ qbar, float* __restrict__ kbar,
+                                                         __nv_bfloat16* __restrict__ qs, __nv_bfloat16* __restrict__ ks) {
+  const long long nsplit = items * D;
   constexpr int V = D / 8;               // vectors per row
   constexpr int G = 256 / V;             // row groups
   constexpr int kMaxIt = MAXR / G;       // rows per thread at block = MAXR
@@ -131,7 +134,15 @@ __global__ void __launch_bounds__(256) block_mean_kernel(const T* __restrict__ q
       float s = 0.f;
 #pragma unroll
       for (int w = 0; w < 8; ++w) s += red[buf][w][c];
-      (c < D ? qbar : kbar)[item * D + (c % D)] = s * inv;
+      const float m = s * inv;
+      float* dst = c < D ? qbar : kbar;        // qbar is NULL when only the terms are wanted
+      if (dst) dst[item * D + (c % D)] = m;
+      __nv_bfloat16* sp = c < D ? qs : ks;
+      if (sp) {
+        const __nv_bfloat16 hi = __float2bfloat16_rn(m);
+        sp[item * D + (c % D)] = hi;
+        sp[nsplit + item * D + (c % D)] = __float2bfloat16_rn(m - __bfloat162float(hi));
+      }
     }
   }
 }
@@ -396,7 +407,7 @@ __global__ void __launch_bounds__(256) combine_partials_kernel(const float2* __r
 // One CTA per resident slot (persistent), from the occupancy of this instantiation.
 template <typename T, int D, int MAXR>
 void launch_mean(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, long long items,
-                 float* qbar, float* kbar, cudaStream_t s) {
+                 float* qbar, float* kbar, cudaStream_t s, void* qs, void* ks) {
   static int per_sm = 0;
   if (!per_sm) {
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, block_mean_kernel<T, D, MAXR>, 256, 0);
@@ -404,13 +415,14 @@ void launch_mean(const void* q, const void* k, const lbsa_qkv_desc& d, int block
   }
   const unsigned grid = static_cast<unsigned>(std::min<long long>(items, static_cast<long long>(per_sm) * num_sms()));
   block_mean_kernel<T, D, MAXR><<<grid, 256, 0, s>>>(static_cast<const T*>(q), static_cast<const T*>(k), d, block,
-                                                     nB, items, qbar, kbar);
+                                                     nB, items, qbar, kbar, static_cast<__nv_bfloat16*>(qs),
+                                                     static_cast<__nv_bfloat16*>(ks));
 }
 
 template <int D>
 cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens, float* scores,
                 void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb, int32_t* status,
-                long long wait_limit, const CUtensorMap* ts) {
+                long long wait_limit, const CUtensorMap* ts, const CUtensorMap* tqs) {
   const long long G = static_cast<long long>(d.B) * d.H;
   float* qbar = static_cast<float*>(ws);
   float* kbar = qbar + G * nB * D;
@@ -418,26 +430,30 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
   const int nQ = tokens ? d.N_valid : nB;
   const int nTk = (nB + kTk - 1) / kTk, nTq = (nQ + kTq - 1) / kTq;
   const long long items = G * nB;
+  // the tensor-core logits take the means as bf16 hi / lo terms, written with the means
+  void *qs = nullptr, *ks = nullptr;
+  const bool tc_tok = tokens && tq && tkb, tc_blk = !tokens && tqs && tkb && ts;
+  if (tc_tok) ks = qbar;                     // the query-block means' slot, unused in this mode
+  if (tc_blk) meanpool_block_split_ptrs(ws, d.B, d.H, nB, D, &qs, &ks);
   if (d.dtype == LBSA_BF16) {
     if (block <= 64)
-      launch_mean<__nv_bfloat16, D, 64>(q, k, d, block, nB, items, qbar, kbar, s);
+      launch_mean<__nv_bfloat16, D, 64>(q, k, d, block, nB, items, tc_tok ? nullptr : qbar, kbar, s, qs, ks);
     else
-      launch_mean<__nv_bfloat16, D, 128>(q, k, d, block, nB, items, qbar, kbar, s);
+      launch_mean<__nv_bfloat16, D, 128>(q, k, d, block, nB, items, tc_tok ? nullptr : qbar, kbar, s, qs, ks);
   } else {
     if (block <= 64)
-      launch_mean<float, D, 64>(q, k, d, block, nB, items, qbar, kbar, s);
+      launch_mean<float, D, 64>(q, k, d, block, nB, items, qbar, kbar, s, qs, ks);
     else
-      launch_mean<float, D, 128>(q, k, d, block, nB, items, qbar, kbar, s);
+      launch_mean<float, D, 128>(q, k, d, block, nB, items, qbar, kbar, s, qs, ks);
   }
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const dim3 lgrid(nTk, nTq, static_cast<unsigned>(G));
   const long long n = static_cast<long long>(nQ) * nB;
   const int chunks = static_cast<int>(std::min<long long>(tokens ? 256 : 64, (n + 2047) / 2048));
-  if (tokens && tq && tkb) {
-    // bf16 token rows: the logits on the tensor cores, from the means' hi / lo terms
-    // (written over the query-block means' slot, which this mode does not use)
-    cudaError_t e = launch_split_means(kbar, G * nB * D, qbar, s);
-    if (e != cudaSuccess) return e;
+  if (tc_tok) {
+    // bf16 token rows: the logits on the tensor cores, from the key means' hi / lo
+    // terms (in the query-block means' slot, which this mode does not use)
+    cudaError_t e;
     const int np = token_logits_parts(nQ, nB);
     TokenLogitsArgs a{static_cast<int>(G), d.H, nQ, nB, D, scale, scores, part, status, wait_limit};
     e = launch_token_logits_bf16(tq, tkb, ts, a, s);
@@ -445,6 +461,16 @@ cudaError_t run(const void* q, const void* k, const lbsa_qkv_desc& d, int block,
     float2* head = part + G * np;
     combine_partials_kernel<<<static_cast<unsigned>(G), 256, 0, s>>>(part, np, head);
     normalize_kernel<<<dim3(chunks, static_cast<unsigned>(G)), 256, 0, s>>>(scores, head, n, 1);
+    return cudaGetLastError();
+  }
+  if (tc_blk) {
+    // both sides are fp32 means: hi / lo terms of each, three chains on the tensor cores
+    cudaError_t e;
+    const int np = token_logits_parts(nQ, nB);
+    TokenLogitsArgs a{static_cast<int>(G), d.H, nQ, nB, D, scale, scores, part, status, wait_limit};
+    e = launch_token_logits_bf16(tqs, tkb, ts, a, s, true);
+    if (e != cudaSuccess) return e;
+    normalize_kernel<<<dim3(chunks, static_cast<unsigned>(G)), 256, 0, s>>>(scores, part, n, np);
     return cudaGetLastError();
   }
   if (!tokens) {
@@ -473,16 +499,26 @@ size_t meanpool_workspace_bytes(int B, int H, int nB, int d, int nQ) {
   const size_t G = static_cast<size_t>(B) * H;
   const size_t nTk = (nB + kTk - 1) / kTk, nTq = (nQ + kTq - 1) / kTq;
   const size_t parts = std::max<size_t>(nTq * nTk, static_cast<size_t>(token_logits_parts(nQ, nB)));
-  return 2 * G * nB * d * sizeof(float) + (G * parts + G) * sizeof(float2) + 256;
+  const size_t base = (2 * G * nB * d * sizeof(float) + (G * parts + G) * sizeof(float2) + 255) / 256 * 256;
+  return base + (nQ == nB ? 2 * G * nB * d * sizeof(float) : 0) + 256;   // + the block proxy's hi / lo terms
+}
+
+void meanpool_block_split_ptrs(void* ws, int B, int H, int nB, int d, void** qs, void** ks) {
+  const size_t G = static_cast<size_t>(B) * H;
+  const size_t nTk = (nB + kTk - 1) / kTk, nTq = (nB + kTq - 1) / kTq;
+  const size_t parts = std::max<size_t>(nTq * nTk, static_cast<size_t>(token_logits_parts(nB, nB)));
+  const size_t base = (2 * G * nB * d * sizeof(float) + (G * parts + G) * sizeof(float2) + 255) / 256 * 256;
+  *qs = static_cast<char*>(ws) + base;
+  *ks = static_cast<char*>(ws) + base + G * nB * d * 2 * sizeof(uint16_t);
 }
 
 void* meanpool_split_ptr(void* ws) { return ws; }   // the query-block means' slot: G x nB x d fp32
 
 cudaError_t launch_meanpool(const void* q, const void* k, const lbsa_qkv_desc& d, int block, int nB, bool tokens,
                             float* scores, void* ws, cudaStream_t s, const CUtensorMap* tq, const CUtensorMap* tkb,
-                            int32_t* status, long long wait_limit, const CUtensorMap* ts) {
-  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts)
-                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts);
+                            int32_t* status, long long wait_limit, const CUtensorMap* ts, const CUtensorMap* tqs) {
+  return d.d == 128 ? run<128>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts, tqs)
+                    : run<64>(q, k, d, block, nB, tokens, scores, ws, s, tq, tkb, status, wait_limit, ts, tqs);
 }
 
 }  // namespace lbsa

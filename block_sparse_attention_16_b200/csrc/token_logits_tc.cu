@@ -9,6 +9,11 @@
 // scores' tolerance once normalised.  Each (128-token tile, 128-key-block
 // chunk) is 2 x d/16 UMMAs of 128 x 128 x 16 into one TMEM accumulator.
 //
+// The block-mean proxy (query-block means against key-block means) runs the
+// same kernel with the query side split the same way (A_SPLIT): then
+//   qbar . kbar = qh . kh + qh . kl + ql . kh   (ql . kl is below 2^-17 of it)
+// three chains into the accumulator, the query rows loaded as two terms.
+//
 // Outputs, as the CUDA-core logits kernel writes them: the scaled logits
 // s_rj into the scores buffer ([g][r][j], fp32) and, per warp of 32 tokens and
 // chunk, the (max, sum of exp(s - max)) of its valid logits, so that the
@@ -24,8 +29,6 @@
 //              UMMAs of chunk c+1 run while the epilogue drains chunk c
 #include <algorithm>
 
-#include <cuda_bf16.h>
-
 #include "lbsa_device.cuh"
 
 namespace lbsa {
@@ -35,12 +38,13 @@ constexpr int kRows = 128;       // tokens per tile
 constexpr int kCols = 128;       // key blocks per chunk
 constexpr int kTLThreads = 192;
 
-template <int D>
+template <int D, bool A_SPLIT>
 struct TLLayout {
-  static constexpr int Q_BYTES = kRows * D * 2;
+  static constexpr int Q_BYTES = kRows * D * 2;            // one term of the query tile
+  static constexpr int NQT = A_SPLIT ? 2 : 1;              // query terms
   static constexpr int TILE_BYTES = kCols * D * 2;        // one term (hi or lo) of one chunk
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RING = Q_BYTES;                 // [stage][term] tiles
+  static constexpr int OFF_RING = NQT * Q_BYTES;           // [stage][term] tiles
   static constexpr int OFF_OUT = OFF_RING + 4 * TILE_BYTES;  // two 128 x 32 fp32 store boxes (16 KB each)
   static constexpr int OUT_BYTES = kRows * 32 * 4;
   static constexpr int OFF_BAR = OFF_OUT + 2 * OUT_BYTES;
@@ -50,11 +54,11 @@ struct TLLayout {
   static constexpr int BYTES = OFF_MISC + 16 + 1024;       // + alignment slack
 };
 
-template <int D, bool TMA_OUT>
+template <int D, bool TMA_OUT, bool A_SPLIT>
 __global__ void __launch_bounds__(kTLThreads, 1)
 token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kb,
                        const __grid_constant__ CUtensorMap tmap_s, const TokenLogitsArgs args) {
-  using L = TLLayout<D>;
+  using L = TLLayout<D, A_SPLIT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -72,7 +76,10 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
 
   const int nTq = (args.nQ + kRows - 1) / kRows;
   const int nC = (args.nB + kCols - 1) / kCols;
-  const long long items = static_cast<long long>(args.G) * nTq;
+  // work items: (head, 128-row tile, group of args.cpi chunks); a small launch
+  // splits a tile's chunks over several CTAs (each loads the tile's query rows)
+  const int nCG = (nC + args.cpi - 1) / args.cpi;
+  const long long items = static_cast<long long>(args.G) * nTq * nCG;
   const long long wl = args.wait_limit;
 
   if (tid == 0) {
@@ -106,14 +113,20 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
       int it = 0, q_loads = 0;
       bool ok = true;
       for (long long item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
-        const int g = static_cast<int>(item / nTq), tq = static_cast<int>(item % nTq);
+        const long long tile = item / nCG;
+        const int g = static_cast<int>(tile / nTq), tq = static_cast<int>(tile % nTq);
+        const int c_lo = static_cast<int>(item % nCG) * args.cpi, c_hi = min(nC, c_lo + args.cpi);
         const int b = g / args.H, h = g % args.H;
         if (it > 0 && !(ok = mbar_wait(q_empty, (it - 1) & 1, wl, args.status, abort_flag))) break;
         ++q_loads;
-        mbar_arrive_expect_tx(q_full, L::Q_BYTES);
-        for (int dc = 0; dc < D / 64; ++dc)
-          tma_load_4d(smem + L::OFF_Q + dc * kRows * 128, &tmap_q, q_full, dc * 64, tq * kRows, h, b);
-        for (int c = 0; c < nC; ++c, ++step) {
+        mbar_arrive_expect_tx(q_full, L::NQT * L::Q_BYTES);
+        for (int u = 0; u < L::NQT; ++u)
+          for (int dc = 0; dc < D / 64; ++dc) {
+            uint8_t* dst = smem + L::OFF_Q + u * L::Q_BYTES + dc * kRows * 128;
+            if (A_SPLIT) tma_load_4d(dst, &tmap_q, q_full, dc * 64, tq * kRows, g, u);   // (d, nQ, G, term)
+            else tma_load_4d(dst, &tmap_q, q_full, dc * 64, tq * kRows, h, b);          // (d, N, H, B)
+          }
+        for (int c = c_lo; c < c_hi; ++c, ++step) {
           const int st = static_cast<int>(step & 1);
           if (step >= 2 && !(ok = mbar_wait(kv_empty + st, ((step >> 1) - 1) & 1, wl, args.status, abort_flag)))
             break;
@@ -141,25 +154,29 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     int it = 0;
     bool ok = true;
     for (long long item = blockIdx.x; ok && item < items; item += gridDim.x, ++it) {
+      const int c_lo = static_cast<int>(item % nCG) * args.cpi, c_hi = min(nC, c_lo + args.cpi);
       if (!(ok = wait0(q_full, it & 1))) break;
-      for (int c = 0; c < nC; ++c, ++step) {
+      for (int c = c_lo; c < c_hi; ++c, ++step) {
         const int st = static_cast<int>(step & 1);
         if (!(ok = wait0(kv_full + st, (step >> 1) & 1))) break;
         if (step >= 2 && !(ok = wait0(acc_empty + st, ((step >> 1) - 1) & 1))) break;
         tc_fence_after();
         if (elect_one()) {
+          // chains (query term, mean term): (0, 0), (0, 1) and, split, (1, 0)
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint64_t b0 = dR + static_cast<uint64_t>(((st * 2 + u) * L::TILE_BYTES) >> 4);
+          for (int ch = 0; ch < (A_SPLIT ? 3 : 2); ++ch) {
+            const int ua = ch == 2 ? 1 : 0, ub = ch == 1 ? 1 : 0;
+            const uint64_t a0 = dQ + static_cast<uint64_t>((ua * L::Q_BYTES) >> 4);
+            const uint64_t b0 = dR + static_cast<uint64_t>(((st * 2 + ub) * L::TILE_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = ((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4;
-              umma_ss(tmem + st * kCols, dQ + off, b0 + off, idesc, (u > 0 || kk > 0) ? 1u : 0u);
+              umma_ss(tmem + st * kCols, a0 + off, b0 + off, idesc, (ch > 0 || kk > 0) ? 1u : 0u);
             }
           }
           umma_commit(kv_empty + st);
           umma_commit(acc_full + st);
-          if (c == nC - 1) umma_commit(q_empty);
+          if (c == c_hi - 1) umma_commit(q_empty);
         }
         __syncwarp();
       }
@@ -174,11 +191,13 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
     long long boxes = 0;                     // TMA store boxes issued (alternating staging buffers)
     bool ok = true;
     for (long long item = blockIdx.x; ok && item < items; item += gridDim.x) {
-      const int g = static_cast<int>(item / nTq), tq = static_cast<int>(item % nTq);
+      const long long tile = item / nCG;
+      const int g = static_cast<int>(tile / nTq), tq = static_cast<int>(tile % nTq);
+      const int c_lo = static_cast<int>(item % nCG) * args.cpi, c_hi = min(nC, c_lo + args.cpi);
       const int row = tq * kRows + warp * 32 + lane;
       const bool rvalid = row < args.nQ;
       float* srow = args.scores + (static_cast<long long>(g) * args.nQ + (rvalid ? row : 0)) * args.nB;
-      for (int c = 0; c < nC; ++c, ++step) {
+      for (int c = c_lo; c < c_hi; ++c, ++step) {
         const int st = static_cast<int>(step & 1);
         // the four warps decide together (they share named barriers below)
         if (!(ok = named_bar_and(2, 128, mbar_wait(acc_full + st, (step >> 1) & 1, wl, args.status, abort_flag))))
@@ -254,17 +273,6 @@ token_logits_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_
   }
 }
 
-// hi = bf16(x), lo = bf16(x - hi) of the fp32 block means, into [2][G][nB][d].
-__global__ void split_means_kernel(const float* __restrict__ kbar, long long n, __nv_bfloat16* __restrict__ out) {
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float x = kbar[i];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    out[i] = hi;
-    out[n + i] = __float2bfloat16_rn(x - __bfloat162float(hi));
-  }
-}
-
 int tl_sms() {
   static int sms = 0;
   if (!sms) {
@@ -280,28 +288,33 @@ int tl_sms() {
 
 int token_logits_parts(int nQ, int nB) { return ((nQ + kRows - 1) / kRows) * ((nB + kCols - 1) / kCols) * 4; }
 
-cudaError_t launch_split_means(const float* kbar, long long n, void* out, cudaStream_t s) {
-  const unsigned grid = static_cast<unsigned>(std::min<long long>((n + 255) / 256, 4L * tl_sms()));
-  split_means_kernel<<<grid, 256, 0, s>>>(kbar, n, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
-}
-
 cudaError_t launch_token_logits_bf16(const CUtensorMap* tq, const CUtensorMap* tkb, const CUtensorMap* ts,
-                                     const TokenLogitsArgs& a, cudaStream_t s) {
+                                     const TokenLogitsArgs& a, cudaStream_t s, bool q_split) {
   if (!(a.d == 64 || a.d == 128) || a.nB < 1 || a.nQ < 1 || a.G < 1) return cudaErrorInvalidValue;
-  const long long items = static_cast<long long>(a.G) * ((a.nQ + kRows - 1) / kRows);
+  const long long tiles = static_cast<long long>(a.G) * ((a.nQ + kRows - 1) / kRows);
+  const int nC = (a.nB + kCols - 1) / kCols;
+  // whole tiles per item, unless that leaves SMs idle: then groups of fewer chunks
+  TokenLogitsArgs b = a;
+  b.cpi = nC;
+  while (b.cpi > 1 && tiles * ((nC + b.cpi - 1) / b.cpi) < tl_sms()) b.cpi = (b.cpi + 1) / 2;
+  const long long items = tiles * ((nC + b.cpi - 1) / b.cpi);
   const unsigned grid = static_cast<unsigned>(std::min<long long>(items, tl_sms()));
   auto go = [&](auto kern, int smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTLThreads, smem, s>>>(*tq, *tkb, ts ? *ts : *tq, a);
+    kern<<<grid, kTLThreads, smem, s>>>(*tq, *tkb, ts ? *ts : *tq, b);
     return cudaGetLastError();
   };
+  if (q_split) {
+    if (!ts) return cudaErrorInvalidValue;
+    return a.d == 128 ? go(token_logits_tc_kernel<128, true, true>, TLLayout<128, true>::BYTES)
+                      : go(token_logits_tc_kernel<64, true, true>, TLLayout<64, true>::BYTES);
+  }
   if (ts)
-    return a.d == 128 ? go(token_logits_tc_kernel<128, true>, TLLayout<128>::BYTES)
-                      : go(token_logits_tc_kernel<64, true>, TLLayout<64>::BYTES);
-  return a.d == 128 ? go(token_logits_tc_kernel<128, false>, TLLayout<128>::BYTES)
-                    : go(token_logits_tc_kernel<64, false>, TLLayout<64>::BYTES);
+    return a.d == 128 ? go(token_logits_tc_kernel<128, true, false>, TLLayout<128, false>::BYTES)
+                      : go(token_logits_tc_kernel<64, true, false>, TLLayout<64, false>::BYTES);
+  return a.d == 128 ? go(token_logits_tc_kernel<128, false, false>, TLLayout<128, false>::BYTES)
+                    : go(token_logits_tc_kernel<64, false, false>, TLLayout<64, false>::BYTES);
 }
 
 }  // namespace lbsa

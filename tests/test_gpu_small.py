@@ -307,6 +307,24 @@ def test_select_head_bit_exact(nB, kind):
 
 
 # ------------------------------------------------------------------ block-mean proxy + head scope
+@pytest.mark.parametrize("d", [128, 64])
+def test_meanpool_scores_on_tensor_cores(d):
+    """Block-mean proxy with bf16 inputs and nB a multiple of 4 (the tensor-core
+    logits): 8,448 tokens, nB = 132 (two 128-row tiles and two 128-column
+    chunks, each 4 wide in the second), every score against the fp64 oracle,
+    head scope bit-exact on them."""
+    wl = small_workload(f"mptc{d}", 1, 2, d, (1, 8, 1056), 64, dtype="bf16", wid=140 + d)
+    assert wl.n_blocks == 132
+    q, k = (x.cuda() for x in make_qkv(wl)[:2])
+    scores = lbsa.lbsa_score(q, k, wl.block, mode="meanpool")
+    bs = lbsa.lbsa_select(scores, wl.block, 0.25, "head")
+    torch.cuda.synchronize()
+    assert lbsa.lbsa_device_status() == 0 and lbsa.lbsa_get_status(bs) == 0
+    sc = host(scores)
+    assert_scores_close(sc, oracle.meanpool_scores(host(q), host(k), wl.n_valid, wl.block))
+    assert_csr_equal(gpu_csr(bs), oracle.select_contract(sc, 0.25, "head"))
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_meanpool_head_scope_pipeline(dtype):
     wl = small_workload("mp", 1, 3, 128, (4, 12, 20), 64, dtype=dtype, wid=140)   # 960 tokens: 15 blocks
