@@ -287,9 +287,12 @@ def test_select_row_bit_exact(nB, kind):
         assert lbsa.lbsa_get_status(bs) == 0
 
 
-@pytest.mark.parametrize("nB", [2, 16, 100, 512])
+@pytest.mark.parametrize("nB", [2, 16, 100, 512, 568, 576])
 @pytest.mark.parametrize("kind", ["softmax", "ties"])
 def test_select_head_bit_exact(nB, kind):
+    """Head scope against the oracle; nB = 568 is the largest the one-launch cluster
+    path holds (71 rows of 568 scores a CTA in shared memory), 576 takes the
+    multi-kernel path."""
     rng = np.random.default_rng(7 + nB)
     H = 2
     if kind == "softmax":
