@@ -27,7 +27,7 @@ __all__ = [
     "lbsa_blockset_info", "lbsa_blockset_export", "lbsa_blockset_from_csr", "lbsa_get_status",
     "lbsa_device_status", "lbsa_partition_perm", "lbsa_permute", "lbsa_selftest_wait", "lbsa_selftest_exp2", "lbsa_select_rule", "lbsa_score_attend",
     "lbsa_select_head_noalloc", "lbsa_select_tokens", "lbsa_select_routed", "lbsa_blockset_views",
-    "lbsa_blockset_masks",
+    "lbsa_blockset_masks", "lbsa_blockset_export_bitmask", "lbsa_blockset_from_bitmask",
     "lbsa_last_error", "lbsa_version", "library_path", "load_library",
     "LBSA_OK", "LBSA_ERR_INVALID_ARG", "LBSA_ERR_UNSUPPORTED", "LBSA_ERR_CUDA", "LBSA_ERR_OOM",
     "LBSA_ERR_BAD_INDEX", "LBSA_ERR_INVALID_SCORES", "LBSA_ERR_TIMEOUT",
@@ -85,6 +85,8 @@ def load_library():
         "lbsa_select_routed": (ctypes.c_int, [P, I32, I32, I32, I32, D, D, I32, P, P, ctypes.POINTER(P), P]),
         "lbsa_blockset_export": (ctypes.c_int, [P, P, P, ctypes.POINTER(I64), P]),
         "lbsa_blockset_from_csr": (ctypes.c_int, [P, P, I32, I32, I32, I32, ctypes.POINTER(P), P]),
+        "lbsa_blockset_export_bitmask": (ctypes.c_int, [P, P, P]),
+        "lbsa_blockset_from_bitmask": (ctypes.c_int, [P, I32, I32, I32, I32, ctypes.POINTER(P), P]),
         "lbsa_get_status": (ctypes.c_int, [P, ctypes.POINTER(I32), I32, P]),
         "lbsa_device_status": (ctypes.c_int, [ctypes.POINTER(I32), I32, P]),
         "lbsa_partition_perm": (ctypes.c_int, [I32, I32, I32, I32, I32, I32, I32, P, I32, P]),
@@ -379,6 +381,32 @@ def lbsa_blockset_from_csr(row_ptr, col, B: int, H: int, nB: int, block: int, st
     _check(load_library().lbsa_blockset_from_csr(_ptr(row_ptr), _ptr(col), B, H, nB, block,
                                                  ctypes.byref(h), _stream(stream)))
     return Blockset(h.value, keep=(row_ptr, col))
+
+
+def lbsa_blockset_export_bitmask(bs: Blockset, stream=None):
+    """The blockset as a block bitmask: int32 [B, H, nB, ceil(nB/32)] on the
+    device (the bits of uint32 words), bit j % 32 of word j // 32 of a row set
+    when key block j is kept."""
+    W = (bs.nB + 31) // 32
+    bits = torch.empty(bs.B, bs.H, bs.nB, W, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
+    _check(load_library().lbsa_blockset_export_bitmask(bs.handle, _ptr(bits), _stream(stream)))
+    return bits
+
+
+def lbsa_blockset_from_bitmask(bits, block: int, stream=None) -> Blockset:
+    """Blockset from a block bitmask on the device, int32 (or uint32 bits)
+    [B, H, nB, ceil(nB/32)] in the layout lbsa_blockset_export_bitmask writes."""
+    if bits.dim() != 4:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "bits must be [B, H, nB, ceil(nB/32)]")
+    B, H, nB, W = bits.shape
+    if W != (nB + 31) // 32:
+        raise LbsaError(LBSA_ERR_INVALID_ARG, f"{W} words a row, ceil(nB/32) = {(nB + 31) // 32} needed")
+    if bits.dtype not in (torch.int32, torch.uint32):
+        raise LbsaError(LBSA_ERR_INVALID_ARG, "bits must be int32 or uint32")
+    _on_device(bits, "bits", bits.dtype, B * H * nB * W)
+    h = ctypes.c_void_p()
+    _check(load_library().lbsa_blockset_from_bitmask(_ptr(bits), B, H, nB, block, ctypes.byref(h), _stream(stream)))
+    return Blockset(h.value, keep=(bits,))
 
 
 def lbsa_get_status(bs: Blockset, clear: bool = False, stream=None) -> int:

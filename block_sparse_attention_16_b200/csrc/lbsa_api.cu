@@ -628,6 +628,35 @@ int lbsa_blockset_from_csr(const int32_t* row_ptr, const int32_t* col, int32_t B
   return LBSA_OK;
 }
 
+int lbsa_blockset_export_bitmask(const lbsa_blockset* bs, uint32_t* bits, void* stream) {
+  if (!bs) return fail(LBSA_ERR_INVALID_ARG, "blockset is NULL");
+  if (!bits) return fail(LBSA_ERR_INVALID_ARG, "bits is NULL");
+  if (bs->masks) return fail(LBSA_ERR_UNSUPPORTED, "per-token blocksets have no block bitmask (use lbsa_blockset_masks)");
+  cudaError_t e = lbsa::launch_export_bitmask(bs, bits, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lbsa_blockset_export_bitmask launch");
+  return LBSA_OK;
+}
+
+int lbsa_blockset_from_bitmask(const uint32_t* bits, int32_t B, int32_t H, int32_t nB, int32_t block,
+                               lbsa_blockset** out, void* stream) {
+  if (!out) return fail(LBSA_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (!bits) return fail(LBSA_ERR_INVALID_ARG, "bits is NULL");
+  if (B < 1 || H < 1 || nB < 1 || nB > 4096) return fail(LBSA_ERR_INVALID_ARG, "bad B/H/nB");
+  if (block != 64 && block != 128) return fail(LBSA_ERR_UNSUPPORTED, "block %d", block);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lbsa_blockset* bs = nullptr;
+  int rc = new_blockset(B, H, nB, block, LBSA_SCOPE_ROW, -1.0, s, &bs);
+  if (rc != LBSA_OK) return rc;
+  cudaError_t e = lbsa::launch_from_bitmask(bits, bs, s);
+  if (e != cudaSuccess) {
+    lbsa_free(bs);
+    return cuda_fail(e, "lbsa_blockset_from_bitmask launch");
+  }
+  *out = bs;
+  return LBSA_OK;
+}
+
 int lbsa_get_status(const lbsa_blockset* bs, int32_t* device_status, int32_t clear, void* stream) {
   if (!bs || !device_status) return fail(LBSA_ERR_INVALID_ARG, "NULL argument");
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -133,6 +133,8 @@ cudaError_t launch_select_tokens(const float* scores, int B, int H, int nQ, int 
                                  void* workspace, cudaStream_t s);
 cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col,
                               int32_t* nnz_dev, cudaStream_t s);
+cudaError_t launch_export_bitmask(const lbsa_blockset* bs, uint32_t* bits, cudaStream_t s);
+cudaError_t launch_from_bitmask(const uint32_t* bits, lbsa_blockset* bs, cudaStream_t s);
 cudaError_t launch_from_csr(const int32_t* row_ptr, const int32_t* col, lbsa_blockset* bs,
                             cudaStream_t s);
 

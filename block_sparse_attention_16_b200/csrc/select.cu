@@ -1023,6 +1023,66 @@ __global__ void from_csr_kernel(const int32_t* __restrict__ row_ptr, const int32
   if (lane == 0) counts[row] = n;
 }
 
+// Block bitmask of a blockset: row r's W = ceil(nB / 32) words, bit j % 32 of
+// word j / 32 set when key block j is kept.  One warp per row: each lane builds
+// its words from the row's ascending ids (a word's ids are a contiguous run).
+__global__ void export_bitmask_kernel(const int32_t* __restrict__ counts, const int32_t* __restrict__ cols, long long R,
+                                      int nB, uint32_t* __restrict__ bits) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;
+  const int W = (nB + 31) >> 5;
+  const int n = counts[row];
+  const int32_t* ids = cols + row * nB;
+  uint32_t* out = bits + row * W;
+  for (int w = lane; w < W; w += 32) out[w] = 0u;
+  __syncwarp();
+  for (int t = lane; t < n; t += 32) {
+    const int j = ids[t];
+    if (j >= 0 && j < nB) atomicOr(out + (j >> 5), 1u << (j & 31));
+  }
+}
+
+// The inverse: ascending ids of the set bits, one warp per row (words in lane
+// order, each lane's ids placed after the lower lanes' by a warp prefix count).
+__global__ void from_bitmask_kernel(const uint32_t* __restrict__ bits, long long R, int nB,
+                                    int32_t* __restrict__ counts, int32_t* __restrict__ cols,
+                                    int32_t* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row >= R) return;
+  const int W = (nB + 31) >> 5;
+  const uint32_t* in = bits + row * W;
+  int32_t* dst = cols + row * nB;
+  const uint32_t tail = (nB & 31) ? ((1u << (nB & 31)) - 1u) : 0xffffffffu;
+  int base = 0;
+  bool bad = false;
+  for (int w0 = 0; w0 < W; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t x = (w < W) ? in[w] : 0u;
+    if (w == W - 1) {
+      bad |= (x & ~tail) != 0u;                 // bits past nB
+      x &= tail;
+    }
+    const int c = __popc(x);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int pos = base + incl - c;
+    while (x) {
+      const int b = __ffs(x) - 1;
+      x &= x - 1;
+      dst[pos++] = w * 32 + b;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(status, LBSA_ERR_BAD_INDEX);
+  if (lane == 0) counts[row] = base;
+}
+
 inline uint32_t fixed_p(double p) {
   return static_cast<uint32_t>(std::nearbyint(p * 16777216.0));   // ties to even in the default mode
 }
@@ -1613,6 +1673,20 @@ cudaError_t launch_export_csr(const lbsa_blockset* bs, int32_t* row_ptr, int32_t
   export_scan_kernel<<<1, 1024, 0, s>>>(bs->counts, R, row_ptr, nnz_dev);
   export_copy_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, s>>>(bs->counts, bs->cols, R, bs->nB,
                                                                                row_ptr, col);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_export_bitmask(const lbsa_blockset* bs, uint32_t* bits, cudaStream_t s) {
+  const long long R = static_cast<long long>(bs->B) * bs->H * bs->nB;
+  export_bitmask_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, s>>>(bs->counts, bs->cols, R, bs->nB,
+                                                                                     bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_from_bitmask(const uint32_t* bits, lbsa_blockset* bs, cudaStream_t s) {
+  const long long R = static_cast<long long>(bs->B) * bs->H * bs->nB;
+  from_bitmask_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, s>>>(bits, R, bs->nB, bs->counts,
+                                                                                   bs->cols, bs->status);
   return cudaGetLastError();
 }
 

@@ -285,6 +285,23 @@ int lbsa_blockset_export(const lbsa_blockset* bs, int32_t* row_ptr, int32_t* col
 int lbsa_blockset_from_csr(const int32_t* row_ptr, const int32_t* col, int32_t B, int32_t H,
                            int32_t nB, int32_t block, lbsa_blockset** out, void* stream);
 
+/* Block bitmask export (the next-row fused dense step's companion format;
+ * ScalingAttention abstract on the mlsift.com sparse-attention listing: a
+ * bit-wise block-sparse mask drives its kernel).  bits: device uint32
+ * [R][W], W = ceil(nB / 32), R = B*H*nB rows as in the blockset; bit (j % 32)
+ * of word j / 32 of row r is set when key block j is kept for row r.  The
+ * caller owns bits.  Asynchronous on `stream`.  Per-token blocksets (whose
+ * entries carry token sets) return LBSA_ERR_UNSUPPORTED. */
+int lbsa_blockset_export_bitmask(const lbsa_blockset* bs, uint32_t* bits, void* stream);
+
+/* Build a blockset from a block bitmask in the layout above (device uint32
+ * [B*H*nB][ceil(nB/32)]), e.g. a static prior mask computed offline.  Copies
+ * the data; the kept ids of each row come out ascending.  Bits past nB in a
+ * row's last word are ignored and raise LBSA_ERR_BAD_INDEX in the status
+ * word. */
+int lbsa_blockset_from_bitmask(const uint32_t* bits, int32_t B, int32_t H, int32_t nB, int32_t block,
+                               lbsa_blockset** out, void* stream);
+
 /* Read (and with clear != 0 reset) the blockset's device status word: 0 or an
  * lbsa_status of the first device error.  Synchronises the stream. */
 int lbsa_get_status(const lbsa_blockset* bs, int32_t* device_status, int32_t clear, void* stream);

@@ -210,3 +210,13 @@ def test_noalloc_head_selection_bounds():
     assert "4096" in lbsa.lbsa_last_error()
     assert lib.lbsa_select_head_noalloc(p, 65535, 65535, 1, 0.25, p, p, p, None) == lbsa.LBSA_ERR_UNSUPPORTED
     assert "B*H=4294836225 heads" in lbsa.lbsa_last_error()
+
+
+def test_bitmask_calls_reject_bad_args():
+    lib = lbsa.load_library()
+    out = ctypes.c_void_p()
+    assert lib.lbsa_blockset_export_bitmask(None, FAKE, None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_blockset_from_bitmask(None, 1, 1, 4, 64, ctypes.byref(out), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4097, 64, ctypes.byref(out), None) == lbsa.LBSA_ERR_INVALID_ARG
+    assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4, 96, ctypes.byref(out), None) == lbsa.LBSA_ERR_UNSUPPORTED
+    assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4, 64, None, None) == lbsa.LBSA_ERR_INVALID_ARG

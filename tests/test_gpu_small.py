@@ -287,6 +287,37 @@ def test_select_row_bit_exact(nB, kind):
         assert lbsa.lbsa_get_status(bs) == 0
 
 
+@pytest.mark.parametrize("nB", [1, 31, 32, 33, 100])
+def test_block_bitmask_round_trip(nB):
+    """Bitmask export sets exactly the kept ids of each row (checked against the
+    oracle's CSR of the same selection); importing it gives the same blockset; a
+    stray bit past nB is dropped and flagged."""
+    rng = np.random.default_rng(90 + nB)
+    x = rng.random((2, 3, nB, nB)).astype(np.float32)
+    x /= x.sum(-1, keepdims=True)
+    s = torch.from_numpy(x).cuda()
+    bs = lbsa.lbsa_select(s, 64, 0.6, "row")
+    bits = lbsa.lbsa_blockset_export_bitmask(bs)
+    torch.cuda.synchronize()
+    rp, col = oracle.select_contract(x, 0.6, "row")
+    W = (nB + 31) // 32
+    words = bits.cpu().numpy().view(np.uint32).reshape(-1, W)
+    for r in range(2 * 3 * nB):
+        want = np.zeros(W, dtype=np.uint32)
+        for j in col[rp[r]:rp[r + 1]]:
+            want[j >> 5] |= np.uint32(1) << np.uint32(j & 31)
+        assert np.array_equal(words[r], want), r
+    back = lbsa.lbsa_blockset_from_bitmask(bits, 64)
+    assert_csr_equal(gpu_csr(back), (rp, col))
+    assert lbsa.lbsa_get_status(back) == 0
+    if nB % 32:
+        stray = bits.clone()
+        stray[0, 0, 0, W - 1] |= torch.tensor(-(1 << 31), dtype=torch.int32, device="cuda")   # bit 31: past nB
+        bad = lbsa.lbsa_blockset_from_bitmask(stray, 64)
+        assert_csr_equal(gpu_csr(bad), (rp, col))
+        assert lbsa.lbsa_get_status(bad) == lbsa.LBSA_ERR_BAD_INDEX
+
+
 @pytest.mark.parametrize("nB", [2, 16, 100, 512, 568, 576])
 @pytest.mark.parametrize("kind", ["softmax", "ties"])
 def test_select_head_bit_exact(nB, kind):
