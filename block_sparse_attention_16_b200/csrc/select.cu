@@ -115,7 +115,16 @@ __global__ void __launch_bounds__(kRowThreads) select_row_kernel(
     tb = mb;
     need = 1;
   } else {
-    uint32_t lo = 0, hi = kInvalidBits;       // invariant: S(lo) >= T > S(hi)
+    // the bracket starts at the weighted scores' range: S(min) = W >= T and S(max + 1) = 0 < T
+    uint32_t bmin = 0xFFFFFFFFu, bmax = 0u;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e)
+      if (wc[e]) {
+        bmin = min(bmin, bits[e]);
+        bmax = max(bmax, bits[e]);
+      }
+    uint32_t lo = __reduce_min_sync(0xffffffffu, bmin);   // invariant: S(lo) >= T > S(hi)
+    uint32_t hi = __reduce_max_sync(0xffffffffu, bmax) + 1u;
     uint64_t S_hi = 0;                        // S(hi)
     uint32_t c_lo = static_cast<uint32_t>(Wc & 2047u), c_hi = 0;   // weighted elements at or above lo / hi
     const uint64_t Tc = T << 11;              // S(mid) >= T  <=>  (S(mid) << 11) + count >= Tc
