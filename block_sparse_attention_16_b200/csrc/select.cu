@@ -617,15 +617,16 @@ __global__ void head_emit_kernel(const float* __restrict__ scores, int G, int nB
 // order from per-row counts and the CTAs' totals; then each warp emits rows.
 // All control flow that spans cluster barriers is uniform over the cluster.
 constexpr int kHC = 8;
-constexpr int kHCT = 512;                     // threads a CTA
+constexpr int kHCT = 1024;                    // threads a CTA (one histogram bin each)
+static_assert(kHCT == kBins, "the digit decision gives each thread one bin");
 constexpr int kHCMaxRows = 2 * kHCT;          // rows a CTA can own
 constexpr int kHCMaxSlice = 40960;            // scores a CTA keeps in shared memory (160 KB)
 
-// S[i] = weight of bins >= 2t + i over the CTA's 1024 bins (kHCT threads x 2)
-__device__ __forceinline__ void hc_suffix(const unsigned long long (&v)[2], unsigned long long (&S)[3],
+// S[i] = weight of bins >= t + i over the CTA's 1024 bins (one a thread)
+__device__ __forceinline__ void hc_suffix(const unsigned long long (&v)[1], unsigned long long (&S)[2],
                                           unsigned long long* warp_tot) {
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  unsigned long long x = v[0] + v[1];
+  unsigned long long x = v[0];
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned long long y = __shfl_down_sync(0xffffffffu, x, o);
@@ -637,7 +638,6 @@ __device__ __forceinline__ void hc_suffix(const unsigned long long (&v)[2], unsi
   for (int u = w + 1; u < kHCT / 32; ++u) later += warp_tot[u];
   S[0] = x + later;
   S[1] = S[0] - v[0];
-  S[2] = S[1] - v[1];
   __syncthreads();                            // warp_tot is reused by the next call
 }
 
@@ -764,13 +764,9 @@ head_select_cluster_kernel(const float* __restrict__ scores, int nQ, int nB, uin
     }
     cl.sync();                                 // every CTA's red is final
     if (search) {
-      unsigned long long v[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int b = 2 * t + i;
-        v[i] = cl.map_shared_rank(red, b / (kBins / kHC))[b % (kBins / kHC)];
-      }
-      unsigned long long S[3];
+      unsigned long long v[1];
+      v[0] = cl.map_shared_rank(red, t / (kBins / kHC))[t % (kBins / kHC)];
+      unsigned long long S[2];
       hc_suffix(v, S, warp_tot);               // (its barriers also publish s_dec[1..2])
       if (pass == 0 && t == 0) {
         if (s_dec[2]) {
@@ -791,9 +787,9 @@ head_select_cluster_kernel(const float* __restrict__ scores, int nQ, int nB, uin
         const unsigned int prefix = s_dec[0];
         __syncthreads();
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 1; ++i) {
           if (above + S[i] >= T && above + S[i + 1] < T) {
-            const unsigned int b = static_cast<unsigned int>(2 * t + i);
+            const unsigned int b = static_cast<unsigned int>(t + i);
             s_state[1] = above + S[i + 1];
             s_dec[0] = (prefix << kDigitBits) | b;
             if (pass == 2) {
