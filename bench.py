@@ -296,13 +296,14 @@ def extra_measurements(lbsa, wl, dev, qp, kp, vp, perm, q, k, v, pk):
     full = torch.full((wl.B, wl.H, nB, nB), 1.0 / nB, device=dev)
     bs1 = lbsa.lbsa_select(full, wl.block, 1.0, "row")
     fd = dense_flops(wl)
-    t_own = _timer(lambda: lbsa.lbsa_attend(qp, kp, vp, bs1))["median"]
+    # LoSA's one dense step (fused dense attention + exact masses, then selection),
+    # timed alternately with our dense attention so that their ratio is free of drift
+    sc_f, o_f = lbsa.lbsa_score_attend(qp, kp, vp, wl.block)
+    t_own, t_fused = _timer_pair(lambda: lbsa.lbsa_attend(qp, kp, vp, bs1),
+                                 lambda: lbsa.lbsa_score_attend(qp, kp, vp, wl.block, scores=sc_f, out=o_f))
     t_sdpa = _timer(lambda: torch.nn.functional.scaled_dot_product_attention(qp, kp, vp))["median"]
     out["dense"] = {"own_p1_ms": t_own, "own_p1_tflops": tf(fd, t_own), "torch_sdpa_ms": t_sdpa,
                     "torch_sdpa_tflops": tf(fd, t_sdpa), "flops": fd}
-    # LoSA's one dense step: fused dense attention + exact masses, then selection
-    sc_f, o_f = lbsa.lbsa_score_attend(qp, kp, vp, wl.block)
-    t_fused = _timer(lambda: lbsa.lbsa_score_attend(qp, kp, vp, wl.block, scores=sc_f, out=o_f))["median"]
     t_sel = _timer(lambda: lbsa.lbsa_select(sc_f, wl.block, P, "row"))["median"]
     sc = lbsa.lbsa_score(qp, kp, wl.block)
     t_score = _timer(lambda: lbsa.lbsa_score(qp, kp, wl.block, scores=sc))["median"]
@@ -688,6 +689,26 @@ def _timer(fn, n=10, warm=3, flush=None):
         ts.append(e0.elapsed_time(e1))
     ts.sort()
     return {"median": ts[len(ts) // 2], "p10": ts[max(0, len(ts) // 10)], "p90": ts[min(len(ts) - 1, (9 * len(ts)) // 10)]}
+
+
+def _timer_pair(fa, fb, n=10, warm=3):
+    """Median device times (ms) of fa() and fb(), timed alternately (a, b, a, b, ...)
+    so that clock drift under the power cap weighs on both alike."""
+    for _ in range(warm):
+        fa()
+        fb()
+    ta, tb = [], []
+    for _ in range(n):
+        for f, ts in ((fa, ta), (fb, tb)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+    ta.sort()
+    tb.sort()
+    return ta[len(ta) // 2], tb[len(tb) // 2]
 
 
 def run_sweep(args):
