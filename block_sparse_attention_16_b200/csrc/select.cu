@@ -902,16 +902,16 @@ __global__ void __launch_bounds__(256) token_emit_kernel(const float* __restrict
     }
     const uint32_t* x = reinterpret_cast<const uint32_t*>(scores) + (static_cast<long long>(g) * nQ + r) * nB;
     uint32_t ties_before = all ? 0u : static_cast<uint32_t>(tiebase[static_cast<long long>(g) * nQ + r]);
-    // eight 32-column loads in flight before the first is used
-    for (int j1 = 0; j1 < nB; j1 += 256) {
-      uint32_t bv[8];
+    // sixteen 32-column loads in flight before the first is used
+    for (int j1 = 0; j1 < nB; j1 += 512) {
+      uint32_t bv[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const int j = j1 + 32 * u + lane;
         bv[u] = (j < nB) ? __ldg(x + j) : 0u;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const int j0 = j1 + 32 * u;
         if (j0 >= nB) break;
         const int j = j0 + lane;
