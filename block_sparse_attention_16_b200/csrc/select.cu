@@ -1335,6 +1335,7 @@ __global__ void __launch_bounds__(256) domain_select_kernel(const float* __restr
                                                             int32_t* __restrict__ cols, int32_t* __restrict__ status) {
   extern __shared__ uint32_t sbits[];         // [M * nB], then M + 1 tie offsets
   __shared__ unsigned long long hist[kBins];
+  __shared__ uint32_t h_lo[kBins], h_hi[kBins];
   __shared__ unsigned long long red[2][8];
   __shared__ uint32_t red_max[8];
   __shared__ unsigned long long s_above;
@@ -1394,25 +1395,39 @@ __global__ void __launch_bounds__(256) domain_select_kernel(const float* __restr
     for (int pass = 0; pass < 3; ++pass) {
       const int shift = 20 - kDigitBits * pass;
 #pragma unroll
-      for (int u = 0; u < kBins / 256; ++u) hist[threadIdx.x + 256 * u] = 0ull;
+      for (int u = 0; u < kBins / 256; ++u) {
+        hist[threadIdx.x + 256 * u] = 0ull;
+        h_lo[threadIdx.x + 256 * u] = 0u;
+        h_hi[threadIdx.x + 256 * u] = 0u;
+      }
       __syncthreads();                        // bins cleared; s_prefix / s_above of the last pass visible
       const uint32_t prefix = s_prefix;
       const unsigned long long above = s_above;
-      // the scores of one row mostly share their high digits: the lanes of a
-      // warp that hit the same bin first add their weights exactly (27 low
-      // bits and the rest, each total < 2^32) and one of them does the atomic
-      for (int e0 = threadIdx.x - lane; e0 < n; e0 += blockDim.x) {   // warp-uniform trip count
-        const int e = e0 + lane;
-        const uint32_t v = (e < n) ? sbits[e] : 0u;
-        const unsigned long long w = (e < n) ? fixed_weight(v) : 0ull;
-        const bool in = w != 0ull && (pass == 0 || (v >> (shift + kDigitBits)) == prefix);
-        const uint32_t bin = in ? ((v >> shift) & (kBins - 1)) : static_cast<uint32_t>(kBins);
-        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-        const uint32_t lo = __reduce_add_sync(peers, static_cast<uint32_t>(w) & ((1u << 27) - 1u));
-        const uint32_t hi = __reduce_add_sync(peers, static_cast<uint32_t>(w >> 27));
-        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (static_cast<unsigned long long>(hi) << 27) + lo);
+      // exact bins: 16 low and 17 high bits of each weight (< 2^33) summed with
+      // 32-bit shared atomics, folded into the 64-bit bins every 2^15 scores so
+      // that neither 32-bit sum can wrap
+      for (int q0 = 0; q0 < n; q0 += 32768) {
+        const int q1 = min(n, q0 + 32768);
+        for (int e = q0 + threadIdx.x; e < q1; e += blockDim.x) {
+          const uint32_t v = sbits[e];
+          if (pass > 0 && (v >> (shift + kDigitBits)) != prefix) continue;
+          const unsigned long long w = fixed_weight(v);
+          if (w) {
+            const uint32_t bin = (v >> shift) & (kBins - 1);
+            atomicAdd(&h_lo[bin], static_cast<uint32_t>(w & 0xFFFFull));
+            atomicAdd(&h_hi[bin], static_cast<uint32_t>(w >> 16));
+          }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kBins / 256; ++u) {
+          const int t = threadIdx.x + 256 * u;
+          hist[t] += (static_cast<unsigned long long>(h_hi[t]) << 16) + h_lo[t];
+          h_lo[t] = 0u;
+          h_hi[t] = 0u;
+        }
+        __syncthreads();
       }
-      __syncthreads();
       // thread t owns bins 4t .. 4t+3: suffix sums S[k] = weight of bins >= 4t + k
       unsigned long long hv[4];
 #pragma unroll
