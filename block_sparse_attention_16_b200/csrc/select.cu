@@ -1137,7 +1137,20 @@ __global__ void __launch_bounds__(256) select_rank_kernel(const float* __restric
   uint32_t tb = 0u;                           // with n == 0 nothing is ranked in
   uint32_t need = 0u;
   if (n > 0) {
-    uint32_t lo = 0, hi = kInvalidBits;       // invariant: cnt(bits >= lo) >= n > cnt(bits >= hi)
+    // the bracket starts at the eligible scores' range: cnt(>= min) = all eligible >= n
+    // and cnt(>= max + 1) = 0 < n; cnt(bits >= hi) is kept as hi moves
+    uint32_t bmin = 0xFFFFFFFFu, bmax = 0u;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const int idx = e * 32 + lane;
+      if (idx < nB && idx != diag) {
+        bmin = min(bmin, bits[e]);
+        bmax = max(bmax, bits[e]);
+      }
+    }
+    uint32_t lo = __reduce_min_sync(0xffffffffu, bmin);   // invariant: cnt(bits >= lo) >= n > cnt(bits >= hi)
+    uint32_t hi = __reduce_max_sync(0xffffffffu, bmax) + 1u;
+    uint32_t c_hi = 0;
     while (hi - lo > 1) {
       const uint32_t mid = lo + ((hi - lo) >> 1);
       uint32_t c = 0;
@@ -1147,18 +1160,15 @@ __global__ void __launch_bounds__(256) select_rank_kernel(const float* __restric
         c += (idx < nB && idx != diag && bits[e] >= mid) ? 1u : 0u;
       }
       c = __reduce_add_sync(0xffffffffu, c);
-      if (c >= static_cast<uint32_t>(n)) lo = mid;
-      else hi = mid;
+      if (c >= static_cast<uint32_t>(n)) {
+        lo = mid;
+      } else {
+        hi = mid;
+        c_hi = c;
+      }
     }
     tb = lo;
-    uint32_t above = 0;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      const int idx = e * 32 + lane;
-      above += (idx < nB && idx != diag && bits[e] > tb) ? 1u : 0u;
-    }
-    above = __reduce_add_sync(0xffffffffu, above);
-    need = static_cast<uint32_t>(n) - above;
+    need = static_cast<uint32_t>(n) - c_hi;   // c_hi = cnt(bits > tb)
   }
   // emit in ascending id order: the own block (mode 0), the ids ranked above tb,
   // and the first `need` ties at tb in id order
