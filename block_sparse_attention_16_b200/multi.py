@@ -110,7 +110,10 @@ def run_sharded_layer(q, k, v, weights, compute, gather: bool = True):
 def attend_units(lbsa, bs, units):
     """The GPU compute of run_sharded_layer: the library's attention on a subset
     of a blockset's (batch, head) units, through a blockset holding only their
-    rows (exported and re-imported as CSR)."""
+    rows (exported and re-imported as CSR).  A rank left without units (more
+    ranks than units) computes nothing and returns an empty [0, N, d] tensor."""
+    if len(units) == 0:
+        return lambda qu, ku, vu, _units: qu[:0]
     row_ptr, col = lbsa.lbsa_blockset_export(bs)
     nB = bs.nB
     rp = row_ptr.to(torch.int64)

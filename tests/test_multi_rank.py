@@ -132,3 +132,44 @@ def test_sharded_layer_on_two_gloo_ranks_equals_one_process(tmp_path):
         assert np.array_equal(np.load(tmp_path / f"full{r}.npy"), ref)
         assert np.load(tmp_path / f"units{r}.npy").tolist() == shards[r]
     assert sorted(shards[0] + shards[1]) == list(range(6)) and shards[0] and shards[1]
+
+
+def test_more_ranks_than_units():
+    """Three ranks, two units: one rank holds none, computes nothing (no library
+    call) and the gather still returns the whole layer on every rank."""
+    from block_sparse_attention_16_b200.multi import attend_units
+    import torch
+    shards = lpt_shards([5.0, 3.0], 3)
+    assert sorted(len(sh) for sh in shards) == [0, 1, 1]
+
+    class NoLibrary:
+        def __getattr__(self, name):
+            raise AssertionError(f"{name} called for a rank without units")
+
+    compute = attend_units(NoLibrary(), None, [])
+    q = torch.zeros(0, 16, 8)
+    assert compute(q, q, q, []).shape == (0, 16, 8)
+
+
+def _uneven_worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import torch
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        B, H, N, d = 1, 2, 8, 4
+        q = torch.arange(B * H * N * d, dtype=torch.float64).reshape(B, H, N, d)
+        out = run_sharded_layer(q, q, q, [2.0, 1.0], lambda qu, ku, vu, units: qu * 2)
+        np.save(os.path.join(out_dir, f"out{rank}.npy"), out.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_layer_with_an_idle_rank(tmp_path):
+    """Three gloo ranks over two units: every rank ends with the whole layer."""
+    import torch
+    mp.start_processes(_uneven_worker, args=(3, _free_port(), str(tmp_path)), nprocs=3, join=True,
+                       start_method="spawn")
+    want = (torch.arange(64, dtype=torch.float64).reshape(1, 2, 8, 4) * 2).numpy()
+    for r in range(3):
+        assert np.array_equal(np.load(tmp_path / f"out{r}.npy"), want)
