@@ -8,6 +8,8 @@ C ABI's names (``include/lbsa.h``):
     bs              = lbsa_select(scores, block, p=0.99, scope="row")
     out             = lbsa_attend(q, k, v, bs)                  # same shape/dtype as q
     row_ptr, col    = lbsa_blockset_export(bs)
+    bits            = lbsa_blockset_export_bitmask(bs)          # [B,H,nB,ceil(nB/32)] block bits
+    scores, out     = lbsa_score_attend(q, k, v, block)          # dense step: O and exact masses
     perm            = lbsa_partition_perm(T, H, W, "3d", tile=(4, 4, 4))
     qp, kp, vp      = lbsa_permute([q, k, v], perm)
 
