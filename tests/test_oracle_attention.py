@@ -32,6 +32,15 @@ def test_dense_matches_torch_sdpa_fp64():
     assert np.max(np.abs(lse - ref_lse)) < 1e-12
 
 
+def test_dense_rows_subset_returns_those_rows():
+    wl, q, k, v = _tiny()
+    O, lse = oracle.dense_attention(q, k, v, wl.n_valid)
+    rows = [7, 2, wl.n_valid - 1]
+    Os, ls = oracle.dense_attention(q, k, v, wl.n_valid, rows=rows)
+    # (a matmul over fewer rows may round in another order: equal to 1e-14)
+    assert np.max(np.abs(Os - O[:, :, rows])) < 1e-14 and np.max(np.abs(ls - lse[:, :, rows])) < 1e-14
+
+
 def test_dense_equal_keys_gives_mean_of_values():
     rng = np.random.default_rng(1)
     q = rng.standard_normal((1, 1, 10, 16))
@@ -107,6 +116,35 @@ def test_sparse_union_of_blocks_matches_sdpa_on_gathered_keys():
         assert np.max(np.abs(O[:, :, i * 16:r1] - ref)) < 1e-12
     # padded rows of the last block stay zero
     assert np.all(O[:, :, wl.n_valid:] == 0)
+
+
+def test_sparse_rows_follow_batch_head_block_order_and_qblocks_subset():
+    # CSR row r = (b*H + h)*nB + i: every (batch, head, query block) has its own
+    # list here, so a row numbered any other way attends to the wrong keys
+    wl = small_workload("t", 2, 3, 16, (2, 5, 7), 16, dtype="f32", wid=305)   # 70 tokens, 5 blocks
+    q, k, v = (x.numpy() for x in make_qkv(wl))
+    B, H, nB, blk = 2, 3, wl.n_blocks, 16
+    rng = np.random.default_rng(8)
+    rows = [np.sort(rng.choice(nB, size=int(rng.integers(1, nB + 1)), replace=False)) for _ in range(B * H * nB)]
+    rp, col = oracle.csr_from_rows(rows)
+    O, lse = oracle.sparse_attention(q, k, v, wl.n_valid, blk, rp, col)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nB):
+                keys = np.concatenate([np.arange(j * blk, min(j * blk + blk, wl.n_valid))
+                                       for j in rows[(b * H + h) * nB + i]])
+                r0, r1 = i * blk, min(i * blk + blk, wl.n_valid)
+                ref = _sdpa64(q[b:b + 1, h:h + 1, r0:r1], k[b:b + 1, h:h + 1, keys], v[b:b + 1, h:h + 1, keys])
+                assert np.max(np.abs(O[b, h, r0:r1] - ref[0, 0])) < 1e-12
+                z = torch.as_tensor(q[b, h, r0:r1], dtype=torch.float64) @ \
+                    torch.as_tensor(k[b, h, keys], dtype=torch.float64).T
+                ref_l = torch.logsumexp(z / math.sqrt(16), dim=-1).numpy()
+                assert np.max(np.abs(lse[b, h, r0:r1] - ref_l)) < 1e-12
+    # a subset of query blocks, in any order, returns those blocks' slices
+    Os, ls = oracle.sparse_attention(q, k, v, wl.n_valid, blk, rp, col, qblocks=[4, 1])
+    assert np.array_equal(Os[:, :, :blk], O[:, :, 4 * blk:5 * blk])
+    assert np.array_equal(Os[:, :, blk:], O[:, :, blk:2 * blk])
+    assert np.array_equal(ls[:, :, blk:], lse[:, :, blk:2 * blk])
 
 
 def test_sparse_empty_row_outputs_zero_and_neg_inf_lse():

@@ -91,6 +91,21 @@ def test_meanpool_matches_torch_pooling_and_softmax():
         assert np.max(np.abs(s[0, h] - ref.numpy())) < 1e-14
 
 
+def test_scores_never_read_padding_rows():
+    # Arrays may be longer than n_valid (a buffer padded to whole blocks); rows
+    # at or past n_valid are not tokens, so filling them with large values must
+    # change no score: the ragged last block holds 9 of 16 tokens here.
+    wl = small_workload("t", 1, 2, 32, (3, 5, 7), 16, dtype="f32")      # 105 tokens, 7 blocks
+    q, k, _ = (x.numpy().astype(np.float64) for x in make_qkv(wl))
+    pad = np.full((1, 2, 7, 32), 1e3)
+    qp, kp = np.concatenate([q, pad], axis=2), np.concatenate([k, -pad], axis=2)
+    assert qp.shape[2] == 112
+    for fn in (oracle.block_mass, oracle.meanpool_scores):
+        a = fn(q, k, wl.n_valid, 16)
+        b = fn(qp, kp, wl.n_valid, 16)
+        assert np.array_equal(a, b), fn.__name__
+
+
 def test_meanpool_zero_keys_uniform():
     q = np.random.default_rng(2).standard_normal((1, 1, 24, 8))
     k = np.zeros((1, 1, 24, 8))

@@ -135,6 +135,27 @@ def test_fixed_point_threshold_values():
     assert oracle.threshold_fixed_point(0.25, 1 << 40) == 1 << 38
 
 
+def test_fractional_weights_are_floored():
+    # Scores below 2^-9 have fp32 bits finer than 2^-32, so their weight
+    # x * 2^32 has a fractional part, which the contract floors.  Hand-worked:
+    # x = (0.25, 0.25, 3 * 2^-34) gives w = (2^30, 2^30, floor(0.75) = 0),
+    # W = 2^31 and, at p = 1/2, T = ceil(2^23 * 2^31 / 2^24) = 2^30, which the
+    # first 0.25 reaches alone.  (Rounded weights would make W = 2^31 + 1 and
+    # T = 2^30 + 1, so both 0.25 blocks; real arithmetic keeps both as well,
+    # since 0.25 < (0.5 + 3 * 2^-34) / 2: the quantum is part of the contract.)
+    tiny = np.float32(3.0 * 2.0 ** -34)
+    assert float(tiny) * 2.0 ** 32 == 0.75
+    x = np.array([[[[0.25, 0.25, tiny]]]], dtype=np.float32)
+    assert _rows(oracle.select_contract(x, 0.5, "row")) == [[0]]
+    assert _rows(oracle.select_fp64(x.astype(np.float64), 0.5, "row")) == [[0, 1]]
+    # scores below the 2^-32 quantum weigh nothing: five 2^-33 (weight
+    # floor(1/2) = 0 each) beside one 2^-20 (weight 2^12) give W = 2^12 and, at
+    # p = 0.999 (P = 16,760,439), T = ceil(P * 2^12 / 2^24) = 4092 <= 2^12
+    y = np.full((1, 1, 1, 6), np.float32(2.0 ** -33), dtype=np.float32)
+    y[0, 0, 0, 4] = np.float32(2.0 ** -20)
+    assert _rows(oracle.select_contract(y, 0.999, "row")) == [[4]]
+
+
 def test_fp64_rule_agrees_on_tiny_workload():
     wl = get_workload("tiny")
     q, k, _ = make_qkv(wl)

@@ -38,6 +38,16 @@ def test_token_scores_match_torch_with_ragged_tail():
     assert np.max(np.abs(s.reshape(2, 2, -1).sum(-1) - 1.0)) < 1e-12
 
 
+def test_token_scores_never_read_padding_rows():
+    # rows at or past n_valid are padding: large values there change no score
+    wl = small_workload("tok", 2, 2, 32, (3, 5, 7), 16, dtype="f32", wid=300)     # 105 tokens, 7 blocks
+    q, k, _ = (x.numpy().astype(np.float64) for x in make_qkv(wl))
+    pad = np.full((2, 2, 7, 32), 1e3)
+    a = oracle.token_meanpool_scores(q, k, wl.n_valid, 16)
+    b = oracle.token_meanpool_scores(np.concatenate([q, pad], 2), np.concatenate([k, -pad], 2), wl.n_valid, 16)
+    assert np.array_equal(a, b)
+
+
 def test_identical_tokens_reduce_to_block_means_over_block_size():
     # every query token of a (full) block equal to the block's mean: the token
     # score matrix repeats each block row `block` times, so it is the
@@ -106,6 +116,28 @@ def test_token_attention_single_block_is_torch_sdpa_over_that_block():
             torch.as_tensor(k[0, 0, keys], dtype=torch.float64)[None],
             torch.as_tensor(v[0, 0, keys], dtype=torch.float64)[None])[0, 0].numpy()
         assert np.max(np.abs(o[0, 0, t] - ref)) < 1e-13
+
+
+def test_token_rows_follow_batch_head_token_order_and_token_subset():
+    # CSR row r = (b*H + h)*n_valid + t, one list per (batch, head, token)
+    wl = small_workload("tokr", 2, 2, 16, (2, 4, 9), 16, dtype="f32", wid=306)   # 72 tokens, 5 blocks
+    q, k, v = (x.numpy() for x in make_qkv(wl))
+    B, H, n, nB = 2, 2, wl.n_valid, 5
+    rng = np.random.default_rng(9)
+    rows = [np.sort(rng.choice(nB, size=int(rng.integers(1, nB + 1)), replace=False)) for _ in range(B * H * n)]
+    rp, col = oracle.csr_from_rows(rows)
+    o, _ = oracle.token_sparse_attention(q, k, v, n, 16, rp, col)
+    for b in range(B):
+        for h in range(H):
+            for t in (0, 17, 40, 71):
+                keys = np.concatenate([np.arange(j * 16, min(j * 16 + 16, n)) for j in rows[(b * H + h) * n + t]])
+                ref = torch.nn.functional.scaled_dot_product_attention(
+                    torch.as_tensor(q[b, h, t:t + 1], dtype=torch.float64)[None],
+                    torch.as_tensor(k[b, h, keys], dtype=torch.float64)[None],
+                    torch.as_tensor(v[b, h, keys], dtype=torch.float64)[None])[0, 0].numpy()
+                assert np.max(np.abs(o[b, h, t] - ref)) < 1e-13
+    sub, _ = oracle.token_sparse_attention(q, k, v, n, 16, rp, col, tokens=[40, 3])
+    assert np.array_equal(sub[:, :, 0], o[:, :, 40]) and np.array_equal(sub[:, :, 1], o[:, :, 3])
 
 
 def _brute_head_select(x32, tau):
