@@ -118,6 +118,11 @@ PLANTED = [
      "head scope: flat index split transposed"),
     (SEL, "select_contract", "_segment_keep(bits[b, h].reshape(-1), w[b, h].reshape(-1), p)",
      "_segment_keep(bits[b, h].T.reshape(-1), w[b, h].T.reshape(-1), p)", "head scope: pairs flattened key-block major"),
+    (SEL, "select_fp64", "if c >= p * total:", "if c > p * total:", "fp64 rule: strict > where it reads >="),
+    (SEL, "select_fp64", "order = np.lexsort((np.arange(n), -seg))", "order = np.lexsort((-np.arange(n), -seg))",
+     "fp64 rule: ties go to the higher index"),
+    (SEL, "csr_from_rows", "row_ptr[r + 1] = row_ptr[r] + len(c)", "row_ptr[r + 1] = len(c)",
+     "CSR offsets not accumulated"),
     # Local + TopK and the per-head floor
     (V, "_order", "np.lexsort((np.arange(n), -bits_row", "np.lexsort((-np.arange(n), -bits_row",
      "ties go to the higher id"),
