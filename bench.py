@@ -929,12 +929,13 @@ def main():
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        # the CPU oracle on rank 0 alone: no process group, no device
+        return run_reference(args, rank, world)
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.impl == "reference":
-            return run_reference(args, rank, world)
         return run_own(args, rank, world)
     finally:
         if world > 1:
