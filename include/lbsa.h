@@ -126,8 +126,10 @@ int lbsa_score(const void* q, const void* k, const lbsa_qkv_desc* desc, int32_t 
  *   scores   out: fp32 [B, H, nB, nB] contiguous, as lbsa_score (exact mode)
  *   out      out: dense attention output, same dtype and strides as q
  *   lse      optional out: fp32 [B, H, N_valid] natural-log row log-sum-exp
- * Scratch: (2 x SM count) strips of (128 + 4) x ceil(N_valid / 64) floats,
- * from the library pool. */
+ * Scratch, from the library pool: one slot per SM of 2 x 128 x
+ * ceil(N_valid / 64) floats (a strip for each row of the two 128-row query
+ * tiles a CTA holds), plus one int32 flag per slot.  nB = ceil(N_valid / block) <= 4096
+ * (LBSA_ERR_UNSUPPORTED beyond). */
 int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qkv_desc* desc, int32_t block,
                       float* scores, void* out, float* lse, void* stream);
 
@@ -149,7 +151,8 @@ int lbsa_score_attend(const void* q, const void* k, const void* v, const lbsa_qk
  * of w is >= T (at least one element).  A segment holding a NaN, negative or
  * >= 2 score keeps all its blocks and sets LBSA_ERR_INVALID_SCORES in the
  * blockset's status word.  The blockset's device memory is allocated
- * stream-ordered at worst-case size (B*H*nB*(nB+1) int32); no host sync. */
+ * stream-ordered at worst-case size (B*H*nB*(nB+1) int32); no host sync.
+ * Limits: nB <= 4096 and B*H*nB < 2^31 (LBSA_ERR_UNSUPPORTED beyond). */
 int lbsa_select(const float* scores, int32_t B, int32_t H, int32_t nB, int32_t block, double p,
                 int32_t scope, lbsa_blockset** out, void* stream);
 
