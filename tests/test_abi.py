@@ -220,3 +220,49 @@ def test_bitmask_calls_reject_bad_args():
     assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4097, 64, ctypes.byref(out), None) == lbsa.LBSA_ERR_INVALID_ARG
     assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4, 96, ctypes.byref(out), None) == lbsa.LBSA_ERR_UNSUPPORTED
     assert lib.lbsa_blockset_from_bitmask(FAKE, 1, 1, 4, 64, None, None) == lbsa.LBSA_ERR_INVALID_ARG
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "lbsa.h"
+
+int main(void) {
+  lbsa_blockset* bs = (lbsa_blockset*)0;
+  lbsa_qkv_desc desc;
+  int rc;
+  memset(&desc, 0, sizeof desc);
+  printf("version %d\n", lbsa_version());
+  rc = lbsa_select((const float*)0, 1, 1, 4, 64, 0.5, LBSA_SCOPE_ROW, &bs, (void*)0);
+  printf("select %d %s\n", rc, lbsa_last_error());
+  rc = lbsa_blockset_from_bitmask((const uint32_t*)0, 1, 1, 4, 64, &bs, (void*)0);
+  printf("from_bitmask %d %s\n", rc, lbsa_last_error());
+  rc = lbsa_attend((const void*)0, (const void*)0, (const void*)0, &desc, bs, (void*)0, (float*)0, (void*)0);
+  printf("attend %d\n", rc);
+  return bs != (lbsa_blockset*)0;
+}
+"""
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    # the boundary is a plain C ABI: a C99 program built with gcc against the
+    # header and the shared library calls it without any Python in between
+    # (argument errors only: they return before any device work)
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    lib_dir = os.path.dirname(lbsa.load_library()._name)
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", lib_dir, "-llbsa", "-Wl,-rpath," + lib_dir],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = r.stdout.splitlines()
+    assert lines[0] == "version 101"
+    assert lines[1].startswith("select 1 ") and "NULL" in lines[1]
+    assert lines[2].startswith("from_bitmask 1 ")
+    assert lines[3] == "attend 1"
