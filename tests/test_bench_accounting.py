@@ -108,3 +108,34 @@ def test_median_entropy_threshold():
     e = np.array([0.39, 0.94, 0.52, 0.83, 0.70, 0.41, 0.9998, 0.9995, 0.9998, 0.9998, 0.9995, 0.9997])
     thr = bench.median_entropy(e)
     assert (e < thr).sum() == 6                           # half the heads pooled
+
+
+def test_traffic_is_reported_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    # profiles/traffic.json holds ncu DRAM bytes with a hash of the kernel's
+    # source files; a changed source must turn the figure into None (null in
+    # the bench line), an unchanged one must give the stored bytes
+    import json
+    import os
+    import shutil
+    d = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    name = next(k for k, v in d.items() if isinstance(v, dict) and "source_hash" in v and bench.load_traffic(k))
+    files = d[name]["files"]
+    (tmp_path / "profiles").mkdir()
+    shutil.copy(os.path.join(bench.ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
+    csrc = tmp_path / "block_sparse_attention_16_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in files:
+        shutil.copy(os.path.join(bench.ROOT, "block_sparse_attention_16_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    before = bench.load_traffic(name)
+    assert before == d[name]["bytes"]
+    with open(csrc / files[0], "a") as fh:
+        fh.write("\n// edited\n")
+    assert bench.load_traffic(name) is None
+    assert bench.load_traffic("no such kernel") is None
+    # the stored figure comes back exactly when the sources are the ones hashed
+    with open(csrc / files[0], "rb") as fh:
+        data = fh.read()
+    with open(csrc / files[0], "wb") as fh:
+        fh.write(data[: -len(b"\n// edited\n")])
+    assert bench.load_traffic(name) == before
