@@ -123,7 +123,7 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def _desc(x: torch.Tensor, n_valid: int | None = None) -> _Desc:
+def _desc(x: torch.Tensor) -> _Desc:
     if x.dim() != 4 or x.stride(-1) != 1:
         raise LbsaError(LBSA_ERR_INVALID_ARG, "expected [B, H, N, d] with a contiguous last dim")
     _on_device(x, "q", contiguous=False)
@@ -134,7 +134,7 @@ def _desc(x: torch.Tensor, n_valid: int | None = None) -> _Desc:
     else:
         raise LbsaError(LBSA_ERR_UNSUPPORTED, f"dtype {x.dtype}")
     B, H, N, d = x.shape
-    return _Desc(B, H, N if n_valid is None else n_valid, d, dt, 0, x.stride(0), x.stride(1), x.stride(2))
+    return _Desc(B, H, N, d, dt, 0, x.stride(0), x.stride(1), x.stride(2))
 
 
 def _on_device(x, name: str, dtype=None, min_numel: int = 0, contiguous: bool = True):
