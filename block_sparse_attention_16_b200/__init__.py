@@ -263,7 +263,8 @@ def lbsa_blockset_masks(bs: Blockset):
 def lbsa_score_attend(q, k, v, block: int, scores=None, out=None, lse=None, want_lse=False, stream=None):
     """Dense attention that also returns the exact block masses (one sweep).
 
-    Returns (scores [B, H, nB, nB] fp32, out) or (scores, out, lse)."""
+    Returns (scores [B, H, nB, nB] fp32, out), or (scores, out, lse) when lse
+    is asked for or given, as lbsa_score does."""
     _same_layout(q, k)
     _same_layout(q, v)
     B, H, N, _ = q.shape
@@ -281,7 +282,7 @@ def lbsa_score_attend(q, k, v, block: int, scores=None, out=None, lse=None, want
     _on_device(lse, "lse", torch.float32, B * H * N)
     _check(load_library().lbsa_score_attend(_ptr(q), _ptr(k), _ptr(v), ctypes.byref(desc), block, _ptr(scores),
                                             _ptr(out), _ptr(lse), _stream(stream)))
-    return (scores, out, lse) if want_lse else (scores, out)
+    return (scores, out, lse) if (want_lse or lse is not None) else (scores, out)
 
 
 _RULES = {"local_topk": 0, "topp_floor": 1}
